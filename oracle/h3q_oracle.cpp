@@ -1,0 +1,304 @@
+// Plain CPU oracle for the INT8 ConvRot (W8A8, Hadamard-256) linear layer.
+//
+// TEST INFRASTRUCTURE ONLY. Only the tests, the package smoke check and the
+// benchmark's CPU-baseline leg may load this library. The product path never
+// calls it and shares no code with it.
+//
+// What it computes, and where the pages state it:
+//  * ConvRot: a group-wise Hadamard rotation along K, expressed as a conv with
+//    kernel = stride = 256, i.e. a block-diagonal product with a 256x256
+//    Hadamard matrix (cloud-worker "MiniMax H3 - research findings", section
+//    "Weight families"; h3-rs README, model-file table: "int8 per-row + ConvRot
+//    (Hadamard-256)").
+//  * Weights stored pre-rotated as per-row int8 with one scale per output row
+//    (h3-rs README, model-file table).
+//  * Activations rotated inside the quantizer and quantized per row (per
+//    token); int8 GEMM; bf16 written directly; SwiGLU fused into fc1's epilogue
+//    (h3-rs README, "Speed", "What makes it fast").
+//  * The FFN-output projection stays INT8 ConvRot, so the SwiGLU output is
+//    rotated and quantized again before it (Minimax_h3_hybrid model card,
+//    "Checkpoints").
+//
+// Readings where the pages are silent (each one is listed with its reason in
+// the design notes): H is the natural-order Sylvester matrix scaled by 1/16; the
+// fp32 sum of each rotated element is a pairwise tree over j in natural order;
+// scale = absmax / 127 (fp32 division); q = clamp(rne(y / scale), -127, 127);
+// one scale per token over the whole row; epilogue order
+// ((float)acc * sx) * sw + bias without fused multiply-add; SwiGLU takes the
+// first half of the fc1 outputs as gate and the second half as up; e^-g is
+// evaluated by Cody-Waite reduction and a degree-7 Taylor polynomial in fp32.
+//
+// Plain loops, no blocking or fusion beyond what the definition states.
+// Build: g++ -O2 -std=c++17 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+extern "C" {
+
+// ---------------------------------------------------------------------------
+// bf16 helpers (bit patterns in uint16_t).
+// ---------------------------------------------------------------------------
+static inline float bf16_to_f32(uint16_t b) {
+  uint32_t u = uint32_t(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+static inline uint16_t f32_to_bf16_rne(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  if ((u & 0x7f800000u) == 0x7f800000u) {            // inf / nan: keep, quiet nan
+    return uint16_t((u >> 16) | ((u & 0xffffu) ? 0x40u : 0u));
+  }
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return uint16_t(u >> 16);
+}
+
+float orc_bf16_to_f32(uint16_t b) { return bf16_to_f32(b); }
+uint16_t orc_f32_to_bf16(float f) { return f32_to_bf16_rne(f); }
+
+// ---------------------------------------------------------------------------
+// Step 1: the 256x256 Hadamard matrix, natural (Sylvester) ordering,
+// H[i][j] = (-1)^popcount(i & j).
+// ---------------------------------------------------------------------------
+static const int kG = 256;
+
+void orc_hadamard256(int8_t* H) {
+  for (int i = 0; i < kG; ++i)
+    for (int j = 0; j < kG; ++j)
+      H[i * kG + j] = (__builtin_popcount(unsigned(i & j)) & 1) ? -1 : 1;
+}
+
+static const std::vector<int8_t>& hadamard() {
+  static std::vector<int8_t> H = [] {
+    std::vector<int8_t> h(kG * kG);
+    orc_hadamard256(h.data());
+    return h;
+  }();
+  return H;
+}
+
+// ---------------------------------------------------------------------------
+// Step 2: rotate each 256-wide group of a row by H/16.
+// y[g*256+i] = sum_j v[g*256+j] * H[i][j] / 16, in fp32. Every term is exact
+// (a sign and a power-of-two scale of the input); the sum is a pairwise tree
+// over j in natural order: level 0 adds terms (2t, 2t+1), level 1 adds those
+// pairs, and so on through level 7.
+// ---------------------------------------------------------------------------
+static void rotate_group_f32(const float* v, float* y) {
+  const std::vector<int8_t>& H = hadamard();
+  float t[kG];
+  for (int i = 0; i < kG; ++i) {
+    for (int j = 0; j < kG; ++j) t[j] = v[j] * (float(H[i * kG + j]) / 16.0f);
+    for (int width = kG; width > 1; width /= 2)
+      for (int p = 0; p < width / 2; ++p) t[p] = t[2 * p] + t[2 * p + 1];
+    y[i] = t[0];
+  }
+}
+
+void orc_rotate_f32(const float* v, int64_t rows, int64_t K, float* y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t g = 0; g < K / kG; ++g)
+      rotate_group_f32(v + r * K + g * kG, y + r * K + g * kG);
+}
+
+// Same rotation in fp64 (plain left-to-right sum), used to check the fp32 one.
+void orc_rotate_f64(const double* v, int64_t rows, int64_t K, double* y) {
+  const std::vector<int8_t>& H = hadamard();
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t g = 0; g < K / kG; ++g)
+      for (int i = 0; i < kG; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < kG; ++j) acc += v[r * K + g * kG + j] * double(H[i * kG + j]);
+        y[r * K + g * kG + i] = acc / 16.0;
+      }
+}
+
+// ---------------------------------------------------------------------------
+// Steps 3-4: per-row symmetric int8 quantization of rotated values.
+// a = max |y| over the whole row; s = a / 127 (fp32); q = clamp(rne(y / s)).
+// A zero row gives s = 0 and q = 0.
+// ---------------------------------------------------------------------------
+static void quantize_row(const float* y, int64_t K, int8_t* q, float* s_out) {
+  float a = 0.0f;
+  for (int64_t k = 0; k < K; ++k) a = std::fmax(a, std::fabs(y[k]));
+  const float s = a / 127.0f;
+  *s_out = s;
+  for (int64_t k = 0; k < K; ++k) {
+    if (s == 0.0f) { q[k] = 0; continue; }
+    float r = std::nearbyint(y[k] / s);   // FE_TONEAREST: ties to even
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    q[k] = int8_t(r);
+  }
+}
+
+void orc_quantize_rows(const float* y, int64_t rows, int64_t K, int8_t* q, float* s) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) quantize_row(y + r * K, K, q + r * K, s + r);
+}
+
+// Activations: bf16 [rows, K] -> rotated int8 [rows, K] + fp32 scale per row.
+void orc_rotate_quant_bf16(const uint16_t* x, int64_t rows, int64_t K, int8_t* q, float* s) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    std::vector<float> v(K), y(K);
+    for (int64_t k = 0; k < K; ++k) v[k] = bf16_to_f32(x[r * K + k]);
+    for (int64_t g = 0; g < K / kG; ++g) rotate_group_f32(v.data() + g * kG, y.data() + g * kG);
+    quantize_row(y.data(), K, q + r * K, s + r);
+  }
+}
+
+// Step 5: weights fp32 [N, K] -> rotated per-row int8 + fp32 scale per row.
+void orc_prepare_weight(const float* w, int64_t N, int64_t K, int8_t* q, float* s) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    std::vector<float> y(K);
+    for (int64_t g = 0; g < K / kG; ++g) rotate_group_f32(w + n * K + g * kG, y.data() + g * kG);
+    quantize_row(y.data(), K, q + n * K, s + n);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Step 6: integer GEMM, acc[m][n] = sum_k xq[m][k] * wq[n][k], exact in int64.
+// Returns the number of entries outside the int32 range (0 expected).
+// ---------------------------------------------------------------------------
+int64_t orc_gemm_s32(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N, int64_t K, int32_t* acc) {
+  int64_t overflow = 0;
+#pragma omp parallel for schedule(static) reduction(+ : overflow)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      int64_t a = 0;
+      for (int64_t k = 0; k < K; ++k) a += int64_t(xq[m * K + k]) * int64_t(wq[n * K + k]);
+      if (a > INT32_MAX || a < INT32_MIN) ++overflow;
+      acc[m * N + n] = int32_t(a);
+    }
+  return overflow;
+}
+
+// ---------------------------------------------------------------------------
+// Step 7: epilogue, v = ((float)acc * sx[m]) * sw[n] (+ bias[n]); out = bf16(v).
+// No fused multiply-add (the build disables contraction).
+// ---------------------------------------------------------------------------
+static inline float epilogue_value(int32_t acc, float sx, float sw, const uint16_t* bias, int64_t n) {
+  float v = float(acc);
+  v = v * sx;
+  v = v * sw;
+  if (bias) v = v + bf16_to_f32(bias[n]);
+  return v;
+}
+
+void orc_epilogue(const int32_t* acc, const float* sx, const float* sw, const uint16_t* bias,
+                  int64_t M, int64_t N, float* v, uint16_t* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      const float x = epilogue_value(acc[m * N + n], sx[m], sw[n], bias, n);
+      if (v) v[m * N + n] = x;
+      if (out) out[m * N + n] = f32_to_bf16_rne(x);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Step 8: SwiGLU, h = silu(g) * u with silu(g) = g / (1 + e^-g).
+// e^t is evaluated in fp32 by Cody-Waite reduction t = n ln2 + r (the two-part
+// ln2 of fdlibm's expf: 0x3f317200 and 0x35bfbe8e), then e^r by the degree-7
+// Taylor polynomial in Horner form with fused multiply-adds, then scaled by 2^n.
+// For t > 88 the value is +inf (silu -> -0); for t < -20, 1 + e^t rounds to 1
+// in fp32 whatever e^t is, so e^t is taken as 0.
+// ---------------------------------------------------------------------------
+float orc_exp_f32(float t) {
+  if (t > 88.0f) return INFINITY;
+  if (t < -20.0f) return 0.0f;
+  const float n = std::nearbyint(t * 1.44269502f);   // log2(e) rounded to fp32
+  float r = std::fma(n, -0.693145751953125f, t);     // ln2 high part (0x3f317200)
+  r = std::fma(n, -1.42860677e-06f, r);              // ln2 low part  (0x35bfbe8e)
+  float p = 1.0f / 5040.0f;
+  p = std::fma(p, r, 1.0f / 720.0f);
+  p = std::fma(p, r, 1.0f / 120.0f);
+  p = std::fma(p, r, 1.0f / 24.0f);
+  p = std::fma(p, r, 1.0f / 6.0f);
+  p = std::fma(p, r, 0.5f);
+  p = std::fma(p, r, 1.0f);
+  p = std::fma(p, r, 1.0f);
+  return std::ldexp(p, int(n));
+}
+
+float orc_silu_f32(float g) { return g / (1.0f + orc_exp_f32(-g)); }
+
+// v [M, 2F] (epilogue values of the fc1 rows: gate = [0,F), up = [F,2F)).
+void orc_swiglu(const float* v, int64_t M, int64_t F, float* h, uint16_t* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t j = 0; j < F; ++j) {
+      const float g = v[m * 2 * F + j];
+      const float u = v[m * 2 * F + F + j];
+      const float x = orc_silu_f32(g) * u;
+      if (h) h[m * F + j] = x;
+      if (out) out[m * F + j] = f32_to_bf16_rne(x);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The layer: x bf16 [M,K] -> rotate+quant -> GEMM with wq [N,K] -> epilogue.
+// epilogue 0: y [M,N]; epilogue 1 (SwiGLU): N = 2F, y [M,F].
+// Optional outputs (nullable): xq, sx, acc, v (fp32 values before bf16).
+// Returns the number of int32 overflows (0 expected).
+// ---------------------------------------------------------------------------
+int64_t orc_linear(const uint16_t* x, int64_t M, int64_t K, const int8_t* wq, const float* sw, int64_t N,
+                   const uint16_t* bias, int epilogue, uint16_t* y,
+                   int8_t* xq_out, float* sx_out, int32_t* acc_out, float* v_out) {
+  std::vector<int8_t> xq(size_t(M) * K);
+  std::vector<float> sx(M);
+  std::vector<int32_t> acc(size_t(M) * N);
+  std::vector<float> v(size_t(M) * N);
+  orc_rotate_quant_bf16(x, M, K, xq.data(), sx.data());
+  const int64_t overflow = orc_gemm_s32(xq.data(), wq, M, N, K, acc.data());
+  orc_epilogue(acc.data(), sx.data(), sw, bias, M, N, v.data(), epilogue == 0 ? y : nullptr);
+  if (epilogue == 1) orc_swiglu(v.data(), M, N / 2, nullptr, y);
+  if (xq_out) std::memcpy(xq_out, xq.data(), xq.size());
+  if (sx_out) std::memcpy(sx_out, sx.data(), sx.size() * 4);
+  if (acc_out) std::memcpy(acc_out, acc.data(), acc.size() * 4);
+  if (v_out) std::memcpy(v_out, v.data(), v.size() * 4);
+  return overflow;
+}
+
+// ---------------------------------------------------------------------------
+// Step 9: FFN, y = down(rotquant(swiglu(gate_up(rotquant(x))))).
+// w_gu [2F, K] (gate rows then up rows), w_down [K, F]. Optional outputs:
+// h (bf16 SwiGLU output [M,F]), hq/sh (its rotated int8 codes and scales).
+// ---------------------------------------------------------------------------
+int64_t orc_ffn(const uint16_t* x, int64_t M, int64_t K, const int8_t* w_gu, const float* s_gu,
+                const uint16_t* b_gu, int64_t F, const int8_t* w_down, const float* s_down,
+                const uint16_t* b_down, uint16_t* y, uint16_t* h_out, int8_t* hq_out, float* sh_out) {
+  std::vector<uint16_t> h(size_t(M) * F);
+  int64_t overflow = orc_linear(x, M, K, w_gu, s_gu, 2 * F, b_gu, 1, h.data(),
+                                nullptr, nullptr, nullptr, nullptr);
+  std::vector<int8_t> hq(size_t(M) * F);
+  std::vector<float> sh(M);
+  overflow += orc_linear(h.data(), M, F, w_down, s_down, K, b_down, 0, y,
+                         hq.data(), sh.data(), nullptr, nullptr);
+  if (h_out) std::memcpy(h_out, h.data(), h.size() * 2);
+  if (hq_out) std::memcpy(hq_out, hq.data(), hq.size());
+  if (sh_out) std::memcpy(sh_out, sh.data(), sh.size() * 4);
+  return overflow;
+}
+
+int orc_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+}  // extern "C"
