@@ -1,0 +1,153 @@
+/*
+ * h3q - INT8 ConvRot (W8A8, Hadamard-256) linear layer for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libh3q.so. The method, as the pages describe it:
+ *  - ConvRot rotation: a group-wise Hadamard rotation along K in 256-wide groups,
+ *    written as a conv whose kernel and stride are the group width
+ *    (cloud-worker "MiniMax H3 - research findings", "Weight families").
+ *  - Weights stored pre-rotated as per-row int8, one scale per output channel
+ *    (h3-rs README, model-file table: "int8 per-row + ConvRot (Hadamard-256)").
+ *  - Activations rotated inside the quantizer and quantized per row (per token);
+ *    an int8 GEMM writes bf16 directly; SwiGLU is fused into the epilogue of the
+ *    FFN's gate/up projection (h3-rs README, "Speed", list "What makes it fast").
+ *  - The FFN-output projection is INT8 ConvRot too (Minimax_h3_hybrid model
+ *    card, "Checkpoints"), so the SwiGLU output is rotated and quantized again.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or retains them. Tensors are row-major and dense
+ *    (leading dimension = width). Every pointer must be 16-byte aligned.
+ *  - bf16 tensors are passed as void* (IEEE bfloat16, 2 bytes per element).
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream); results are
+ *    ready when the stream reaches that point.
+ *  - Arguments are checked on the host before anything is launched; a failed
+ *    check returns H3Q_ERR_INVALID_ARG (or H3Q_ERR_UNSUPPORTED for a valid
+ *    shape outside the implemented range) and launches nothing.
+ *  - A launch failure returns H3Q_ERR_CUDA. A device-side bounded wait that ran
+ *    out (it never should) is reported later by h3q_get_device_status.
+ *  - H = natural-order Sylvester Hadamard matrix, H[i][j] = (-1)^popcount(i&j),
+ *    applied as H/16 (orthonormal). Each rotated element is an fp32 sum whose
+ *    order is fixed (radix-2 butterflies over index bits 0,1,...,7), so the
+ *    int8 codes are reproducible bit for bit.
+ *  - Quantizer: s = max|y| / 127 per row (fp32 division), q = clamp(rne(y / s),
+ *    -127, 127); an all-zero row gives s = 0 and q = 0.
+ */
+#ifndef H3Q_H_
+#define H3Q_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  H3Q_OK = 0,
+  H3Q_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or workspace: nothing launched */
+  H3Q_ERR_UNSUPPORTED = 2,  /* valid request outside the implemented range: nothing launched */
+  H3Q_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  H3Q_ERR_TIMEOUT = 4       /* a bounded device wait expired (reported by h3q_get_device_status) */
+} h3q_status;
+
+enum { H3Q_EPI_NONE = 0, H3Q_EPI_SWIGLU = 1 };
+
+/* Largest K (or F) the rotate+quantize kernel holds on chip for one row. */
+#define H3Q_MAX_K 32768
+
+/*
+ * Rotate + per-token quantize (h3-rs README, "What makes it fast": the ConvRot
+ * Hadamard rotation is done warp-level inside the quantizer, activations are
+ * quantized per row).
+ *   x_bf16 [M, K] bf16 in; xq [M, K] int8 out (rotated codes); sx [M] fp32 out.
+ *   K % 256 == 0, 256 <= K <= H3Q_MAX_K; M >= 1 (M == 0 is a no-op).
+ */
+h3q_status h3q_rotate_quant(const void* x_bf16, int64_t M, int64_t K, int8_t* xq, float* sx,
+                            cudaStream_t stream);
+
+/*
+ * Offline weight preparation (h3-rs README, model-file table: int8 per-row +
+ * ConvRot): rotate each fp32 row along K by the same block-diagonal H/16, then
+ * per-row int8 with one fp32 scale per output channel.
+ *   w [N, K] fp32 in; wq [N, K] int8 out; sw [N] fp32 out. Same K rules as above.
+ */
+h3q_status h3q_prepare_weight(const float* w, int64_t N, int64_t K, int8_t* wq, float* sw,
+                              cudaStream_t stream);
+
+/*
+ * W8A8 linear with fused epilogue (h3-rs README, "What makes it fast": the fused
+ * int8 GEMM writes bf16 directly; fc1's SwiGLU fuses into its epilogue).
+ *   acc[m][n] = sum_k xq[m][k] * wq[n][k] (exact int32);
+ *   v = ((float)acc * sx[m]) * sw[n] (+ bias[n]), fp32, no fused multiply-add.
+ *   epilogue H3Q_EPI_NONE:   y [M, N] bf16 = bf16_rne(v).
+ *   epilogue H3Q_EPI_SWIGLU: N = 2F, rows [0, F) of wq are the gate, [F, 2F) the
+ *     up projection; y [M, F] bf16 = bf16_rne(silu(v_gate) * v_up), silu(g) =
+ *     g / (1 + e^-g) with e^-g from Cody-Waite reduction and a degree-7 Taylor
+ *     polynomial in fp32.
+ *   xq [M, K] int8, sx [M] fp32 (from h3q_rotate_quant); wq [N, K] int8, sw [N]
+ *   fp32 (from h3q_prepare_weight); bias_bf16 [N] bf16 or NULL.
+ *   K % 256 == 0; N % 8 == 0 (SwiGLU: F % 128 == 0); M >= 1.
+ */
+h3q_status h3q_linear_w8a8(const int8_t* xq, const float* sx, int64_t M, int64_t K,
+                           const int8_t* wq, const float* sw, int64_t N,
+                           const void* bias_bf16, int epilogue, void* y_bf16, cudaStream_t stream);
+
+/*
+ * FFN block, INT8 ConvRot end to end (h3-rs README "What makes it fast";
+ * Minimax_h3_hybrid model card, "Checkpoints": the FFN-output projection stays
+ * INT8 ConvRot and the SwiGLU path stays fused):
+ *   y [M, K] = down( rotquant( swiglu( gate_up( rotquant(x) ) ) ) ).
+ *   x_bf16 [M, K]; w_gu [2F, K] int8 with s_gu [2F] (gate rows, then up rows);
+ *   b_gu [2F] bf16 or NULL; w_down [K, F] int8 with s_down [K]; b_down [K] bf16
+ *   or NULL; y_bf16 [M, K] out.
+ *   workspace: caller-owned device scratch of at least
+ *   h3q_ffn_workspace_size(M, K, F) bytes, 256-byte aligned (holds xq, sx,
+ *   h, hq, sh). K % 256 == 0, F % 256 == 0, K, F <= H3Q_MAX_K.
+ */
+size_t h3q_ffn_workspace_size(int64_t M, int64_t K, int64_t F);
+h3q_status h3q_ffn(const void* x_bf16, int64_t M, int64_t K,
+                   const int8_t* w_gu, const float* s_gu, const void* b_gu, int64_t F,
+                   const int8_t* w_down, const float* s_down, const void* b_down,
+                   void* y_bf16, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Test hook: the same GEMM kernel with the raw int32 accumulators as output.
+ *   xq [M, K], wq [N, K] int8; acc [M, N] int32. K % 128 == 0, N % 8 == 0.
+ */
+h3q_status h3q_gemm_s32(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N, int64_t K,
+                        int32_t* acc, cudaStream_t stream);
+
+/*
+ * Synchronizes `stream`, then reports and clears the device status word:
+ * H3Q_ERR_TIMEOUT if any bounded wait in a kernel of this library ran out since
+ * the last call, H3Q_ERR_CUDA if the synchronization failed, else H3Q_OK.
+ */
+h3q_status h3q_get_device_status(cudaStream_t stream);
+
+/*
+ * Upper bound, in nanoseconds, on every spin-wait inside the GEMM kernel (an
+ * mbarrier the kernel waits on). Past it the kernel records H3Q_ERR_TIMEOUT,
+ * drains its own copies in flight (again bounded), frees its tensor memory and
+ * returns. Default 2 s. Values below 1000 ns are raised to 1000 ns.
+ */
+void h3q_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Test hook for the bounded-wait path: launches one block that waits on an
+ * mbarrier nothing ever arrives on, with the given limit; afterwards
+ * h3q_get_device_status returns H3Q_ERR_TIMEOUT. No fault, no hang.
+ */
+h3q_status h3q_test_stalled_wait(uint64_t limit_ns, cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* h3q_status_string(h3q_status s);
+
+/* Library version string (static). */
+const char* h3q_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3Q_H_ */

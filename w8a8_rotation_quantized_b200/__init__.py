@@ -1,0 +1,133 @@
+"""INT8 ConvRot (W8A8, Hadamard-256) linear layer on B200: Python binding of libh3q.so.
+
+The functions carry the C ABI's names (include/h3q.h) and only marshal
+arguments: torch tensors in device memory become pointers, the current CUDA
+stream becomes the stream argument, and a non-OK status raises H3QError. Every
+step of the computation runs in the library's kernels. There is no fallback:
+if the library is missing or cannot be loaded, importing this package fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libh3q.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "h3q.h")
+
+H3Q_OK, H3Q_ERR_INVALID_ARG, H3Q_ERR_UNSUPPORTED, H3Q_ERR_CUDA, H3Q_ERR_TIMEOUT = range(5)
+H3Q_EPI_NONE, H3Q_EPI_SWIGLU = 0, 1
+H3Q_MAX_K = 32768
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python w8a8_rotation_quantized_b200/build.py` "
+                      "(or __graft_entry__.build())")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_P, _I64, _SZ, _INT, _U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int, ctypes.c_uint64
+_SIGS = {
+    "h3q_rotate_quant": (_INT, [_P, _I64, _I64, _P, _P, _P]),
+    "h3q_prepare_weight": (_INT, [_P, _I64, _I64, _P, _P, _P]),
+    "h3q_linear_w8a8": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _INT, _P, _P]),
+    "h3q_ffn_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "h3q_ffn": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]),
+    "h3q_gemm_s32": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P]),
+    "h3q_get_device_status": (_INT, [_P]),
+    "h3q_set_wait_limit_ns": (None, [_U64]),
+    "h3q_test_stalled_wait": (_INT, [_U64, _P]),
+    "h3q_status_string": (ctypes.c_char_p, [_INT]),
+    "h3q_version": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype, _fn.argtypes = _res, _args
+
+
+class H3QError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.h3q_status_string(status).decode()} (status {status})")
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/h3q.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(h3q_\w+)\s*\(", text, flags=re.M)))
+
+
+def _check(status: int, where: str) -> None:
+    if status != H3Q_OK:
+        raise H3QError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def h3q_rotate_quant(x, xq, sx, stream=None) -> None:
+    """x bf16 [M, K] -> xq int8 [M, K] (rotated codes), sx fp32 [M]."""
+    M, K = x.shape
+    _check(lib.h3q_rotate_quant(_ptr(x), M, K, _ptr(xq), _ptr(sx), _stream(stream)), "h3q_rotate_quant")
+
+
+def h3q_prepare_weight(w, wq, sw, stream=None) -> None:
+    """w fp32 [N, K] -> wq int8 [N, K] (rotated along K), sw fp32 [N]."""
+    N, K = w.shape
+    _check(lib.h3q_prepare_weight(_ptr(w), N, K, _ptr(wq), _ptr(sw), _stream(stream)), "h3q_prepare_weight")
+
+
+def h3q_linear_w8a8(xq, sx, wq, sw, y, bias=None, epilogue=H3Q_EPI_NONE, stream=None) -> None:
+    """y bf16 = rescale(xq @ wq^T) (+ bias); SwiGLU epilogue: y [M, N/2]."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    _check(lib.h3q_linear_w8a8(_ptr(xq), _ptr(sx), M, K, _ptr(wq), _ptr(sw), N, _ptr(bias), int(epilogue),
+                               _ptr(y), _stream(stream)), "h3q_linear_w8a8")
+
+
+def h3q_ffn_workspace_size(M: int, K: int, F: int) -> int:
+    return int(lib.h3q_ffn_workspace_size(M, K, F))
+
+
+def h3q_ffn(x, w_gu, s_gu, w_down, s_down, y, workspace, b_gu=None, b_down=None, stream=None) -> None:
+    """y [M, K] = down(rotquant(swiglu(gate_up(rotquant(x)))))."""
+    M, K = x.shape
+    F = w_gu.shape[0] // 2
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.h3q_ffn(_ptr(x), M, K, _ptr(w_gu), _ptr(s_gu), _ptr(b_gu), F, _ptr(w_down), _ptr(s_down),
+                       _ptr(b_down), _ptr(y), _ptr(workspace), nbytes, _stream(stream)), "h3q_ffn")
+
+
+def h3q_gemm_s32(xq, wq, acc, stream=None) -> None:
+    """acc int32 [M, N] = xq [M, K] @ wq [N, K]^T."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    _check(lib.h3q_gemm_s32(_ptr(xq), _ptr(wq), M, N, K, _ptr(acc), _stream(stream)), "h3q_gemm_s32")
+
+
+def h3q_get_device_status(stream=None) -> int:
+    return int(lib.h3q_get_device_status(_stream(stream)))
+
+
+def h3q_set_wait_limit_ns(ns: int) -> None:
+    lib.h3q_set_wait_limit_ns(int(ns))
+
+
+def h3q_test_stalled_wait(limit_ns: int, stream=None) -> None:
+    _check(lib.h3q_test_stalled_wait(int(limit_ns), _stream(stream)), "h3q_test_stalled_wait")
+
+
+def h3q_status_string(status: int) -> str:
+    return lib.h3q_status_string(int(status)).decode()
+
+
+def h3q_version() -> str:
+    return lib.h3q_version().decode()

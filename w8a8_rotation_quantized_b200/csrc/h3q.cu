@@ -1,0 +1,231 @@
+// libh3q.so: the C ABI declared in include/h3q.h. Host-side argument checks,
+// TMA descriptor setup and launches of the kernels in rotquant.cuh and
+// gemm_sm100.cuh. Everything is stream-ordered; nothing here allocates device
+// memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "h3q.h"
+#include "gemm_sm100.cuh"
+#include "rotquant.cuh"
+
+namespace {
+
+using h3q::GemmParams;
+
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [rows, cols] int8 row-major, boxes of 128 columns x 128 rows, 128-byte swizzle;
+// reads past the edges return zeros.
+bool make_tmap_i8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+template <int EPI>
+h3q_status launch_gemm(const int8_t* a, const int8_t* b, int64_t M, int64_t K, int64_t b_rows, int64_t N_out,
+                       const float* sx, const float* sw, const void* bias, void* out, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  if (!make_tmap_i8(&ta, a, M, K) || !make_tmap_i8(&tb, b, b_rows, K)) return H3Q_ERR_CUDA;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(h3q::gemm_i8_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(h3q::kGemmSmem));
+  });
+  if (attr_err != cudaSuccess) return H3Q_ERR_CUDA;
+  GemmParams p;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N_out);
+  p.K = static_cast<int>(K);
+  p.num_m = static_cast<int>((M + h3q::kBM - 1) / h3q::kBM);
+  p.num_n = (EPI == h3q::kEpiSwiGLU) ? static_cast<int>(N_out / 128)
+                                     : static_cast<int>((N_out + h3q::kBN - 1) / h3q::kBN);
+  p.num_tiles = p.num_m * p.num_n;
+  p.b_row_up = (EPI == h3q::kEpiSwiGLU) ? static_cast<int>(N_out) : 0;
+  p.sx = sx;
+  p.sw = sw;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.out = out;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const int sms = sm_count();
+  if (sms <= 0) return H3Q_ERR_CUDA;
+  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  h3q::gemm_i8_kernel<EPI><<<grid, h3q::kGemmThreads, h3q::kGemmSmem, stream>>>(ta, tb, p);
+  return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+}
+
+bool valid_k(int64_t K) { return K >= 256 && K % 256 == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct FfnLayout {
+  size_t xq, sx, h, hq, sh, total;
+};
+
+FfnLayout ffn_layout(int64_t M, int64_t K, int64_t F) {
+  FfnLayout l;
+  size_t off = 0;
+  l.xq = off; off = align256(off + size_t(M) * size_t(K));
+  l.sx = off; off = align256(off + size_t(M) * 4);
+  l.h = off;  off = align256(off + size_t(M) * size_t(F) * 2);
+  l.hq = off; off = align256(off + size_t(M) * size_t(F));
+  l.sh = off; off = align256(off + size_t(M) * 4);
+  l.total = off;
+  return l;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* h3q_version(void) { return "h3q 0.1 (sm_100a, tcgen05 int8)"; }
+
+const char* h3q_status_string(h3q_status s) {
+  switch (s) {
+    case H3Q_OK: return "ok";
+    case H3Q_ERR_INVALID_ARG: return "invalid argument";
+    case H3Q_ERR_UNSUPPORTED: return "unsupported shape";
+    case H3Q_ERR_CUDA: return "CUDA error";
+    case H3Q_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+void h3q_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns < 1000 ? 1000 : ns); }
+
+h3q_status h3q_rotate_quant(const void* x_bf16, int64_t M, int64_t K, int8_t* xq, float* sx,
+                            cudaStream_t stream) {
+  if (M < 0 || !valid_k(K)) return H3Q_ERR_INVALID_ARG;
+  if (M == 0) return H3Q_OK;
+  if (!x_bf16 || !xq || !sx || !aligned16(x_bf16) || !aligned16(xq) || !aligned16(sx)) return H3Q_ERR_INVALID_ARG;
+  if (K > H3Q_MAX_K || M > INT32_MAX) return H3Q_ERR_UNSUPPORTED;
+  const cudaError_t e = h3q::launch_rotquant(static_cast<const __nv_bfloat16*>(x_bf16), M, K, xq, sx, stream);
+  return e == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+}
+
+h3q_status h3q_prepare_weight(const float* w, int64_t N, int64_t K, int8_t* wq, float* sw, cudaStream_t stream) {
+  if (N < 0 || !valid_k(K)) return H3Q_ERR_INVALID_ARG;
+  if (N == 0) return H3Q_OK;
+  if (!w || !wq || !sw || !aligned16(w) || !aligned16(wq) || !aligned16(sw)) return H3Q_ERR_INVALID_ARG;
+  if (K > H3Q_MAX_K || N > INT32_MAX) return H3Q_ERR_UNSUPPORTED;
+  const cudaError_t e = h3q::launch_rotquant(w, N, K, wq, sw, stream);
+  return e == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+}
+
+h3q_status h3q_linear_w8a8(const int8_t* xq, const float* sx, int64_t M, int64_t K, const int8_t* wq,
+                           const float* sw, int64_t N, const void* bias_bf16, int epilogue, void* y_bf16,
+                           cudaStream_t stream) {
+  if (M < 0 || !valid_k(K) || N <= 0 || N % 8 != 0) return H3Q_ERR_INVALID_ARG;
+  if (epilogue != H3Q_EPI_NONE && epilogue != H3Q_EPI_SWIGLU) return H3Q_ERR_INVALID_ARG;
+  if (epilogue == H3Q_EPI_SWIGLU && (N % 256 != 0)) return H3Q_ERR_INVALID_ARG;  // F = N/2 multiple of 128
+  if (M == 0) return H3Q_OK;
+  if (!xq || !sx || !wq || !sw || !y_bf16) return H3Q_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(sx) || !aligned16(wq) || !aligned16(sw) || !aligned16(y_bf16) ||
+      (bias_bf16 && !aligned16(bias_bf16)))
+    return H3Q_ERR_INVALID_ARG;
+  if (M > INT32_MAX - 256 || N > INT32_MAX - 512 || K > INT32_MAX) return H3Q_ERR_UNSUPPORTED;
+  if (epilogue == H3Q_EPI_SWIGLU)
+    return launch_gemm<h3q::kEpiSwiGLU>(xq, wq, M, K, N, N / 2, sx, sw, bias_bf16, y_bf16, stream);
+  return launch_gemm<h3q::kEpiBF16>(xq, wq, M, K, N, N, sx, sw, bias_bf16, y_bf16, stream);
+}
+
+h3q_status h3q_gemm_s32(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N, int64_t K, int32_t* acc,
+                        cudaStream_t stream) {
+  if (M < 0 || N <= 0 || N % 8 != 0 || K < 128 || K % 128 != 0) return H3Q_ERR_INVALID_ARG;
+  if (M == 0) return H3Q_OK;
+  if (!xq || !wq || !acc || !aligned16(xq) || !aligned16(wq) || !aligned16(acc)) return H3Q_ERR_INVALID_ARG;
+  if (M > INT32_MAX - 256 || N > INT32_MAX - 512 || K > INT32_MAX) return H3Q_ERR_UNSUPPORTED;
+  return launch_gemm<h3q::kEpiS32>(xq, wq, M, K, N, N, nullptr, nullptr, nullptr, acc, stream);
+}
+
+size_t h3q_ffn_workspace_size(int64_t M, int64_t K, int64_t F) {
+  if (M < 0 || K <= 0 || F <= 0) return 0;
+  return ffn_layout(M, K, F).total;
+}
+
+h3q_status h3q_ffn(const void* x_bf16, int64_t M, int64_t K, const int8_t* w_gu, const float* s_gu,
+                   const void* b_gu, int64_t F, const int8_t* w_down, const float* s_down, const void* b_down,
+                   void* y_bf16, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (M < 0 || !valid_k(K) || !valid_k(F)) return H3Q_ERR_INVALID_ARG;
+  if (M == 0) return H3Q_OK;
+  if (!x_bf16 || !w_gu || !s_gu || !w_down || !s_down || !y_bf16 || !workspace) return H3Q_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(w_gu) || !aligned16(s_gu) || !aligned16(w_down) || !aligned16(s_down) ||
+      !aligned16(y_bf16) || (b_gu && !aligned16(b_gu)) || (b_down && !aligned16(b_down)) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return H3Q_ERR_INVALID_ARG;
+  if (K > H3Q_MAX_K || F > H3Q_MAX_K || M > INT32_MAX - 256) return H3Q_ERR_UNSUPPORTED;
+  const FfnLayout l = ffn_layout(M, K, F);
+  if (workspace_bytes < l.total) return H3Q_ERR_INVALID_ARG;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + l.xq);
+  float* sx = reinterpret_cast<float*>(ws + l.sx);
+  void* h = ws + l.h;
+  int8_t* hq = reinterpret_cast<int8_t*>(ws + l.hq);
+  float* sh = reinterpret_cast<float*>(ws + l.sh);
+  h3q_status st = h3q_rotate_quant(x_bf16, M, K, xq, sx, stream);
+  if (st != H3Q_OK) return st;
+  st = h3q_linear_w8a8(xq, sx, M, K, w_gu, s_gu, 2 * F, b_gu, H3Q_EPI_SWIGLU, h, stream);
+  if (st != H3Q_OK) return st;
+  st = h3q_rotate_quant(h, M, F, hq, sh, stream);
+  if (st != H3Q_OK) return st;
+  return h3q_linear_w8a8(hq, sh, M, F, w_down, s_down, K, b_down, H3Q_EPI_NONE, y_bf16, stream);
+}
+
+h3q_status h3q_get_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return H3Q_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, h3q::g_status, sizeof(v)) != cudaSuccess) return H3Q_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(h3q::g_status, &zero, sizeof(zero)) != cudaSuccess) return H3Q_ERR_CUDA;
+    return H3Q_ERR_TIMEOUT;
+  }
+  return H3Q_OK;
+}
+
+h3q_status h3q_test_stalled_wait(uint64_t limit_ns, cudaStream_t stream) {
+  if (limit_ns > 10000000000ull) return H3Q_ERR_INVALID_ARG;  // at most 10 s
+  h3q::stalled_wait_kernel<<<1, 32, 0, stream>>>(limit_ns < 1000 ? 1000 : limit_ns);
+  return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+}
+
+}  // extern "C"
