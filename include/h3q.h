@@ -54,7 +54,7 @@ typedef enum {
 enum { H3Q_EPI_NONE = 0, H3Q_EPI_SWIGLU = 1 };
 
 /* Largest K (or F) the rotate+quantize kernel holds on chip for one row. */
-#define H3Q_MAX_K 32768
+#define H3Q_MAX_K 16384
 
 /*
  * Rotate + per-token quantize (h3-rs README, "What makes it fast": the ConvRot

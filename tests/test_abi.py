@@ -55,7 +55,7 @@ def test_rotate_quant_rejects(args):
 
 
 def test_rotate_quant_too_wide_is_unsupported():
-    assert h3q.lib.h3q_rotate_quant(FAKE, 4, 32768 + 256, FAKE, FAKE, None) == h3q.H3Q_ERR_UNSUPPORTED
+    assert h3q.lib.h3q_rotate_quant(FAKE, 4, 16384 + 256, FAKE, FAKE, None) == h3q.H3Q_ERR_UNSUPPORTED
 
 
 def test_zero_rows_is_a_noop():

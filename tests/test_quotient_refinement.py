@@ -1,0 +1,20 @@
+"""The rotate+quantize kernel forms y / s as a reciprocal product refined twice
+with fused multiply-add residuals (Markstein's correction). This checks, in C on
+the host with IEEE fp32 arithmetic (the same correctly rounded operations the
+GPU executes), that the scheme returns exactly the IEEE quotient, including
+dividends a few ulps from the half-integer points where the int8 code is
+decided."""
+import os
+import subprocess
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def test_refined_quotient_equals_ieee_division(tmp_path):
+    exe = tmp_path / "quotient_check"
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-o", str(exe),
+                           os.path.join(HERE, "csrc", "quotient_check.c"), "-lm"])
+    out = subprocess.run([str(exe), "2000", "20000"], capture_output=True, text=True, check=True)
+    bad, cases = map(int, out.stdout.split())
+    assert cases == 40_000_000
+    assert bad == 0, out.stderr

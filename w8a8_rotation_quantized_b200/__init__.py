@@ -18,7 +18,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "h3q.h")
 
 H3Q_OK, H3Q_ERR_INVALID_ARG, H3Q_ERR_UNSUPPORTED, H3Q_ERR_CUDA, H3Q_ERR_TIMEOUT = range(5)
 H3Q_EPI_NONE, H3Q_EPI_SWIGLU = 0, 1
-H3Q_MAX_K = 32768
+H3Q_MAX_K = 16384
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python w8a8_rotation_quantized_b200/build.py` "
