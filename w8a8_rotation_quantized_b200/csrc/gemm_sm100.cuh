@@ -6,26 +6,35 @@
 //
 //   acc[m][n] = sum_k A[m][k] * B[n][k]     A = xq [M, K], B = wq [N, K], both K-major
 //
-// Design (one CTA per SM, persistent):
-//   warp 0      TMA producer: one 128x128 int8 box of A and two of B per stage
-//               into a STAGES-deep ring of 128-byte-swizzled shared memory.
-//   warp 1      allocates 512 TMEM columns; one lane issues 4 MMAs of
-//               128 x 256 x 32 per stage and commits each stage back to the
-//               producer and each finished tile to the epilogue.
-//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter of the
-//               accumulator, fp32 rescale, bias, bf16 (or SwiGLU), stores.
+// Design (persistent; CTA pairs, one CTA per SM; cta_group::2 MMAs):
+//   A pair computes 256 x 256 output tiles: CTA r holds rows 128r .. 128r+127
+//   of the A tile and rows 128r .. 128r+127 of the B tile, and the pair's
+//   M=256 MMA (issued by the leader, rank 0) reads both CTAs' shared memory, so
+//   each SM stages half the operand bytes a one-SM 128 x 256 tile would need.
+//   warp 0      TMA producer (both CTAs): one 128x128 int8 box of A and one of B
+//               per stage into a STAGES-deep ring of 128-byte-swizzled shared
+//               memory; both CTAs' boxes complete on the leader's full barrier.
+//   warp 1      allocates 512 TMEM columns (pair allocation); in the leader one
+//               lane issues 4 MMAs of 256 x 256 x 32 per stage and commits each
+//               stage back to both producers and each finished tile to both
+//               epilogues.
+//   warps 2-9   epilogue (both CTAs): each warp takes a 32-lane quarter of the
+//               CTA's 128 accumulator rows and half of the columns; the tile's
+//               column scales and biases are staged in shared memory first;
+//               tcgen05.ld, fp32 rescale, bias, bf16 (or SwiGLU), stores; then
+//               they free the accumulator on the leader's barrier.
 // Two 256-column accumulators let the epilogue of tile i overlap the main loop
 // of tile i+1. Tiles are walked in groups of GROUP_M row blocks so the weight
-// blocks in flight stay in L2.
+// blocks in flight stay in L2. No load uses cluster multicast.
 //
 // SwiGLU: the B tile of an output tile holding h columns [j0, j0+128) stacks
-// gate rows [j0, j0+128) over up rows [F+j0, F+j0+128) of the plain [gate; up]
-// weight, so one 128 x 256 accumulator holds both halves and silu(g) * u is
-// formed per element in the epilogue. This gives the locality that the pages get
+// gate rows [j0, j0+128) (in the leader) over up rows [F+j0, F+j0+128) (in the
+// peer) of the plain [gate; up] weight, so each CTA's 128 x 256 accumulator
+// holds both halves and silu(g) * u is formed per element in the epilogue. This gives the locality that the pages get
 // by interleaving gate/up rows at load, without repacking the weight.
 //
-// Every wait is bounded (see mbar_wait_bounded); past the limit the block
-// records a timeout, drains its own copies and MMAs (bounded again), frees its
+// Every wait is bounded (see mbar_wait_bounded); past the limit the pair
+// records a timeout, drains its copies and MMAs (bounded again), frees its
 // tensor memory and exits.
 #pragma once
 
@@ -37,16 +46,17 @@
 
 namespace h3q {
 
-constexpr int kBM = 128;
-constexpr int kBN = 256;
+constexpr int kBM = 128;  // rows per CTA; a CTA pair computes 256-row tiles
+constexpr int kBN = 256;  // output columns per tile; each CTA holds 128 rows of B
 constexpr int kBK = 128;  // int8 elements = 128 bytes = one swizzle row
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kAStage = kBM * kBK;  // 16 KB
-constexpr int kBStage = kBN * kBK;  // 32 KB
+constexpr int kBStage = 128 * kBK;  // 16 KB: this CTA's half of the B tile
 constexpr int kTmemCols = 512;
-constexpr int kGemmThreads = 192;
-constexpr int kGroupM = 16;
-constexpr size_t kGemmSmem = size_t(kStages) * (kAStage + kBStage) + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kGemmThreads = 320;  // producer, MMA, 8 epilogue warps
+constexpr int kGroupM = 8;  // pair tiles (256 rows each) per raster group
+constexpr size_t kGemmSmem =
+    size_t(kStages) * (kAStage + kBStage) + 1024 /*align*/ + 256 /*barriers*/ + 4 * kBN * 4 /*column scales, biases*/;
 
 enum EpiKind : int { kEpiS32 = 0, kEpiBF16 = 1, kEpiSwiGLU = 2 };
 
@@ -80,7 +90,11 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int&
 __device__ __forceinline__ float exp_f32(float t) {
   if (t > 88.0f) return __int_as_float(0x7F800000);
   if (t < -20.0f) return 0.0f;
-  const float n = rintf(__fmul_rn(t, 1.44269502f));
+  // n = rne(t log2 e): adding 1.5 * 2^23 rounds to an integer (ties to even) and
+  // leaves it in the low mantissa bits
+  const float nm = __fadd_rn(__fmul_rn(t, 1.44269502f), 12582912.0f);
+  const float n = __fsub_rn(nm, 12582912.0f);
+  const int ni = __float_as_int(nm) - 0x4B400000;
   float r = __fmaf_rn(n, -0.693145751953125f, t);
   r = __fmaf_rn(n, -1.42860677e-06f, r);
   float p = 1.0f / 5040.0f;
@@ -91,7 +105,7 @@ __device__ __forceinline__ float exp_f32(float t) {
   p = __fmaf_rn(p, r, 0.5f);
   p = __fmaf_rn(p, r, 1.0f);
   p = __fmaf_rn(p, r, 1.0f);
-  return __fmul_rn(p, __int_as_float((static_cast<int>(n) + 127) << 23));
+  return __fmul_rn(p, __int_as_float((ni + 127) << 23));
 }
 
 __device__ __forceinline__ float silu_f32(float g) { return __fdiv_rn(g, __fadd_rn(1.0f, exp_f32(-g))); }
@@ -101,23 +115,6 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) { return __ui
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// Loads 8 consecutive fp32 values and 8 bf16 values (as fp32) starting at n.
-__device__ __forceinline__ void load_col8(const float* sw, const __nv_bfloat16* bias, int n, float (&s)[8],
-                                          float (&b)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(sw + n));
-  const float4 c = __ldg(reinterpret_cast<const float4*>(sw + n) + 1);
-  s[0] = a.x; s[1] = a.y; s[2] = a.z; s[3] = a.w; s[4] = c.x; s[5] = c.y; s[6] = c.z; s[7] = c.w;
-  if (bias != nullptr) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(bias + n));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      b[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
-      b[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
-    }
-  }
 }
 
 // v = ((float)acc * sx) * sw (+ bias), no fused multiply-add.
@@ -130,10 +127,12 @@ __device__ __forceinline__ float rescale(uint32_t acc_bits, float sxr, float swn
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
+  // identical offsets in both CTAs of the pair: the leader's MMA addresses the
+  // peer's operand tiles through the same shared-memory offsets
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kAStage;
@@ -144,19 +143,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* col_scale = reinterpret_cast<float*>(smem + kStages * (kAStage + kBStage) + 256);  // [2][kBN]
+  float* col_bias = col_scale + 2 * kBN;                                                      // [2][kBN]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader: issues the pair's MMAs
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int KB = p.K / kBK;
   const uint64_t limit = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&full[s], 1);   // leader's: its expect_tx; both CTAs' boxes complete on it
+      mbar_init(&empty[s], 1);  // the leader's MMA commit
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tfull[b], 1);   // the leader's MMA commit
+      mbar_init(&tempty[b], 16);  // leader's: 8 epilogue warps of each CTA
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -167,36 +170,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------------------ producer
+      // ------------------------------------------------------------ producer (both CTAs)
       const uint64_t pol = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
         int mb, nb;
         tile_coords(tile, p.num_m, p.num_n, mb, nb);
-        const int b_row0 = (EPI == kEpiSwiGLU) ? nb * 128 : nb * kBN;
-        const int b_row1 = (EPI == kEpiSwiGLU) ? p.b_row_up + nb * 128 : nb * kBN + 128;
+        const int a_row = mb * (2 * kBM) + static_cast<int>(rank) * kBM;
+        const int b_row = (EPI == kEpiSwiGLU) ? (rank == 0 ? nb * 128 : p.b_row_up + nb * 128)
+                                              : nb * kBN + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, limit, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], kAStage + kBStage);
-          tma_load_2d(sA + stage * kAStage, &tmA, &full[stage], kb * kBK, mb * kBM, pol);
-          tma_load_2d(sB + stage * kBStage, &tmB, &full[stage], kb * kBK, b_row0, pol);
-          tma_load_2d(sB + stage * kBStage + kBStage / 2, &tmB, &full[stage], kb * kBK, b_row1, pol);
+          const uint32_t full_leader = cluster_map(&full[stage], 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (kAStage + kBStage));
+          tma_load_2d_pair(sA + stage * kAStage, &tmA, full_leader, kb * kBK, a_row, pol);
+          tma_load_2d_pair(sB + stage * kBStage, &tmB, full_leader, kb * kBK, b_row, pol);
           ++issued;
           if (++stage == kStages) {
             stage = 0;
@@ -204,8 +208,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (!ok) {
-        // drain this block's own copies still in flight (bounded, ignores abort)
+      if (!ok && rank == 0) {
+        // drain the pair's copies still in flight (bounded, ignores abort)
         for (int s = 0; s < kStages; ++s) {
           if (issued <= s) continue;
           const long last = ((issued - 1 - s) / kStages) * kStages + s;
@@ -214,16 +218,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_i8(kBM, kBN);
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------------ MMA issuer (leader only)
+      constexpr uint32_t idesc = idesc_i8(2 * kBM, kBN);
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
       uint32_t buf_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-        if (!mbar_wait_bounded(&tempty[buf], buf_phase ^ 1u, limit, abort_flag)) break;
+      for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
+        if (!mbar_wait_bounded_cluster(&tempty[buf], buf_phase ^ 1u, limit, abort_flag)) break;
         tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(buf * kBN);
         for (int kb = 0; kb < KB; ++kb) {
@@ -237,42 +241,67 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int k = 0; k < kBK / 32; ++k) {
             // advance the start address by 32 bytes (= 2 in 16-byte units) per K step
-            mma_i8(d, ad + 2u * k, bd + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            mma_i8_pair(d, ad + 2u * k, bd + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
           }
-          mma_commit(&empty[stage]);
+          mma_commit_pair(cluster_map(&empty[stage], 0));
+          mma_commit_pair(cluster_map(&empty[stage], 1));
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(&tfull[buf]);
+        mma_commit_pair(cluster_map(&tfull[buf], 0));
+        mma_commit_pair(cluster_map(&tfull[buf], 1));
         buf ^= 1;
         if (buf == 0) buf_phase ^= 1u;
       }
-      // every MMA this block issued has completed once `drain` fires
-      mma_commit(drain);
+      // every MMA this pair issued has completed once `drain` fires
+      mma_commit_pair(cluster_map(drain, 0));
       mbar_wait_bounded(drain, 0, limit, nullptr);
     }
   } else {
-    // -------------------------------------------------------------- epilogue
-    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 belong to this warp
-    const int row_in_tile = quarter * 32 + lane;
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    // Warps 2..9: warp w reads TMEM lanes 32*(w%4) .. +31 (its quarter of the
+    // CTA's 128 rows) and one half of the tile's columns.
+    const int quarter = warp & 3;
+    const int chalf = (warp - 2) >> 2;
+    const int et = threadIdx.x - 64;  // 0 .. 255
+    const int row_in_tile = static_cast<int>(rank) * kBM + quarter * 32 + lane;
+    const uint32_t tempty_leader0 = cluster_map(&tempty[0], 0);
+    const uint32_t tempty_leader1 = cluster_map(&tempty[1], 0);
+    const bool has_bias = p.bias != nullptr;
     int buf = 0;
     uint32_t buf_phase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    int iter = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++iter) {
       int mb, nb;
       tile_coords(tile, p.num_m, p.num_n, mb, nb);
-      if (!mbar_wait_bounded(&tfull[buf], buf_phase, limit, abort_flag)) break;
+      float* cs = col_scale + (iter & 1) * kBN;  // this tile's 256 column scales ...
+      float* cb = col_bias + (iter & 1) * kBN;   // ... and biases, staged once per tile
+      if constexpr (EPI != kEpiS32) {
+        int n;
+        bool valid;
+        if constexpr (EPI == kEpiSwiGLU) {
+          n = et < 128 ? nb * 128 + et : p.b_row_up + nb * 128 + (et - 128);
+          valid = true;
+        } else {
+          n = nb * kBN + et;
+          valid = n < p.N;
+        }
+        cs[et] = valid ? __ldg(p.sw + n) : 0.0f;
+        cb[et] = (valid && has_bias) ? __bfloat162float(p.bias[n]) : 0.0f;
+        named_barrier(1, 256);
+      }
+      if (!mbar_wait_bounded_cluster(&tfull[buf], buf_phase, limit, abort_flag)) break;
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * kBN);
-      const int row = mb * kBM + row_in_tile;
+      const int row = mb * (2 * kBM) + row_in_tile;
       const bool row_ok = row < p.M;
-
       if constexpr (EPI == kEpiS32) {
         int32_t* out = static_cast<int32_t*>(p.out) + static_cast<int64_t>(row) * p.N;
 #pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = 4 * chalf; c < 4 * chalf + 4; ++c) {
           uint32_t r[32];
           tmem_ld32(taddr + c * 32, r);
           tmem_ld_wait();
@@ -290,25 +319,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       } else if constexpr (EPI == kEpiBF16) {
         const float sxr = row_ok ? __ldg(p.sx + row) : 0.0f;
-        const bool has_bias = p.bias != nullptr;
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.N;
 #pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = 4 * chalf; c < 4 * chalf + 4; ++c) {
           uint32_t r[32];
           tmem_ld32(taddr + c * 32, r);
           tmem_ld_wait();
-          const int n0 = nb * kBN + c * 32;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            const int n = n0 + 8 * g;
+            const int i0 = c * 32 + 8 * g;  // column within the tile
+            const int n = nb * kBN + i0;
             if (n < p.N) {
-              float s[8], b[8];
-              load_col8(p.sw, p.bias, n, s, b);
               uint32_t o[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                const float v0 = rescale(r[8 * g + 2 * i], sxr, s[2 * i], b[2 * i], has_bias);
-                const float v1 = rescale(r[8 * g + 2 * i + 1], sxr, s[2 * i + 1], b[2 * i + 1], has_bias);
+                const int k = i0 + 2 * i;
+                const float v0 = rescale(r[8 * g + 2 * i], sxr, cs[k], cb[k], has_bias);
+                const float v1 = rescale(r[8 * g + 2 * i + 1], sxr, cs[k + 1], cb[k + 1], has_bias);
                 o[i] = pack_bf16x2(v0, v1);
               }
               if (row_ok) *reinterpret_cast<uint4*>(out + n) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -317,41 +344,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       } else {  // SwiGLU: accumulator columns [0,128) gate, [128,256) up
         const float sxr = row_ok ? __ldg(p.sx + row) : 0.0f;
-        const bool has_bias = p.bias != nullptr;
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.N;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 2 * chalf; c < 2 * chalf + 2; ++c) {
           uint32_t rg[32], ru[32];
           tmem_ld32(taddr + c * 32, rg);
           tmem_ld32(taddr + 128 + c * 32, ru);
           tmem_ld_wait();
-          const int j0 = nb * 128 + c * 32;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            const int j = j0 + 8 * g;
-            float sg[8], bg[8], su[8], bu[8];
-            load_col8(p.sw, p.bias, j, sg, bg);
-            load_col8(p.sw, p.bias, p.b_row_up + j, su, bu);
+            const int i0 = c * 32 + 8 * g;  // gate column within the tile; up column is 128 + i0
             uint32_t o[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               float h[2];
 #pragma unroll
               for (int e = 0; e < 2; ++e) {
-                const int k = 2 * i + e;
-                const float gv = rescale(rg[8 * g + k], sxr, sg[k], bg[k], has_bias);
-                const float uv = rescale(ru[8 * g + k], sxr, su[k], bu[k], has_bias);
+                const int k = i0 + 2 * i + e;
+                const float gv = rescale(rg[8 * g + 2 * i + e], sxr, cs[k], cb[k], has_bias);
+                const float uv = rescale(ru[8 * g + 2 * i + e], sxr, cs[128 + k], cb[128 + k], has_bias);
                 h[e] = __fmul_rn(silu_f32(gv), uv);
               }
               o[i] = pack_bf16x2(h[0], h[1]);
             }
-            if (row_ok) *reinterpret_cast<uint4*>(out + j) = make_uint4(o[0], o[1], o[2], o[3]);
+            if (row_ok) *reinterpret_cast<uint4*>(out + nb * 128 + i0) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (lane == 0) mbar_arrive_cluster(buf == 0 ? tempty_leader0 : tempty_leader1);
       buf ^= 1;
       if (buf == 0) buf_phase ^= 1u;
     }
@@ -359,9 +381,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // the leader's MMAs read the peer's shared memory: both stay until all are done
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
 }
 
 // Test kernel for the bounded-wait path: waits on an mbarrier that nothing ever

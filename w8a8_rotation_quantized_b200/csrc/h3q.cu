@@ -76,7 +76,7 @@ h3q_status launch_gemm(const int8_t* a, const int8_t* b, int64_t M, int64_t K, i
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N_out);
   p.K = static_cast<int>(K);
-  p.num_m = static_cast<int>((M + h3q::kBM - 1) / h3q::kBM);
+  p.num_m = static_cast<int>((M + 2 * h3q::kBM - 1) / (2 * h3q::kBM));  // 256-row tiles of a CTA pair
   p.num_n = (EPI == h3q::kEpiSwiGLU) ? static_cast<int>(N_out / 128)
                                      : static_cast<int>((N_out + h3q::kBN - 1) / h3q::kBN);
   p.num_tiles = p.num_m * p.num_n;
@@ -88,7 +88,8 @@ h3q_status launch_gemm(const int8_t* a, const int8_t* b, int64_t M, int64_t K, i
   p.wait_limit_ns = g_wait_limit_ns.load();
   const int sms = sm_count();
   if (sms <= 0) return H3Q_ERR_CUDA;
-  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  const int pairs = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
+  const int grid = 2 * pairs;  // clusters of two CTAs
   h3q::gemm_i8_kernel<EPI><<<grid, h3q::kGemmThreads, h3q::kGemmSmem, stream>>>(ta, tb, p);
   return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
 }
@@ -138,7 +139,8 @@ h3q_status h3q_rotate_quant(const void* x_bf16, int64_t M, int64_t K, int8_t* xq
   if (M == 0) return H3Q_OK;
   if (!x_bf16 || !xq || !sx || !aligned16(x_bf16) || !aligned16(xq) || !aligned16(sx)) return H3Q_ERR_INVALID_ARG;
   if (K > H3Q_MAX_K || M > INT32_MAX) return H3Q_ERR_UNSUPPORTED;
-  const cudaError_t e = h3q::launch_rotquant(static_cast<const __nv_bfloat16*>(x_bf16), M, K, xq, sx, stream);
+  const cudaError_t e = h3q::launch_rotquant(static_cast<const __nv_bfloat16*>(x_bf16), M, K, xq, sx,
+                                             g_wait_limit_ns.load(), stream);
   return e == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
 }
 
@@ -147,7 +149,7 @@ h3q_status h3q_prepare_weight(const float* w, int64_t N, int64_t K, int8_t* wq, 
   if (N == 0) return H3Q_OK;
   if (!w || !wq || !sw || !aligned16(w) || !aligned16(wq) || !aligned16(sw)) return H3Q_ERR_INVALID_ARG;
   if (K > H3Q_MAX_K || N > INT32_MAX) return H3Q_ERR_UNSUPPORTED;
-  const cudaError_t e = h3q::launch_rotquant(w, N, K, wq, sw, stream);
+  const cudaError_t e = h3q::launch_rotquant(w, N, K, wq, sw, g_wait_limit_ns.load(), stream);
   return e == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
 }
 

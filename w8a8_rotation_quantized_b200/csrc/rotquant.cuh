@@ -2,93 +2,82 @@
 // quantizer (h3-rs README, "What makes it fast"), followed by per-row
 // (per-token) absmax int8 quantization.
 //
-// Layout: a half-warp (16 lanes) owns one 256-group; lane l of the half holds
-// elements 16l .. 16l+15, loaded with 16-byte accesses (one half-warp reads 512
-// contiguous bytes of bf16). Index bits 0-3 live in registers, bits 4-7 are the
-// lane bits. The Walsh-Hadamard butterflies run in ascending bit order: bits
-// 0-2 on packed fp32 pairs (v[r], v[r+8]) with the sm_100 two-wide fp32 adds,
-// bit 3 inside each pair, bits 4-7 across lanes by shuffles. Every butterfly is
-// one correctly rounded fp32 add or subtract, so each rotated value has the same
-// bits as the pairwise-tree sum of the explicit H/16 product. The 1/16 moves to
-// the scale: y16 = 16 y and s16 = max|y16| / 127 = 16 s exactly, and
-// y16 / s16 = y / s, so the codes are unchanged.
+// Data movement: a persistent grid; in each block one producer thread streams
+// work items (R whole rows, contiguous in memory) into a ring of shared-memory
+// stages with 1D bulk copies (cp.async.bulk, completion on an mbarrier), so
+// several items are in flight per block while the consumer warps work. Each row
+// is read from HBM once and its codes written once.
 //
-// Quantization needs rne(RN(y / s)) for every element. Instead of a division per
-// element, each row gets rs = RN(1 / s) once, and each quotient is formed by
-// q0 = RN(y rs) refined twice with exact FMA residuals, e = y - q s,
-// q <- RN(q + e rs) (Markstein, "Computation of elementary functions on the IBM
-// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): after the first
-// step q is within one ulp of y/s, and then the second step returns the
-// correctly rounded quotient. Rows whose scale is below 2^-100 (never met in
-// practice) fall back to IEEE division. The integer is read from the bits of
-// q + 1.5*2^23, whose add rounds half to even; its low byte is the int8 code.
+// Work split: a half-warp (16 lanes) of the consumers owns one 256-group of a
+// row. Lane l of the half reads two 16-byte runs of the group from shared
+// memory: elements 8l .. 8l+7 and 128+8l .. 128+8l+7 (bank-conflict free), kept
+// as packed pairs p[r] = (v[r], v[r+8]) of element 8l+r and 128+8l+r. Index bits
+// 0-2 are register bits, bits 3-6 the lane bits, bit 7 the pair half.
+//
+// Rotation: the unnormalized Walsh-Hadamard butterflies in ascending index-bit
+// order: bits 0-2 on packed pairs with the sm_100 two-wide fp32 add, bits 3-6
+// across lanes by shuffles (a fused multiply by +-1 and add, one rounding),
+// bit 7 inside each pair. Every butterfly is one correctly rounded fp32 add or
+// subtract, so each rotated value has the same bits as the pairwise-tree sum of
+// the explicit H/16 product. The 1/16 moves to the scale: y16 = 16 y and
+// s16 = max|y16| / 127 = 16 s exactly, and y16 / s16 = y / s, so the codes are
+// unchanged.
+//
+// Quantization needs rne(RN(y / s)) per element. Each row gets rs = RN(1/s)
+// once; each quotient is q0 = RN(y rs) refined twice with exact FMA residuals,
+// e = y - q s, q <- RN(q + e rs) (Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990): after the first step q is within one ulp of y/s, and the second step
+// returns the correctly rounded quotient. Rows whose scale is below 2^-100
+// (never met in practice) use IEEE division. The integer is read from the bits
+// of q + 1.5*2^23, whose add rounds half to even; its low byte is the int8 code.
 // |y| <= max|y| bounds y/s by 127 (1 + 2^-23), so no clamp is needed.
-//
-// Work item = R whole rows (all their groups), held on chip until each row's
-// absmax is known: one pass over HBM. The grid is persistent and each block
-// loads its next item while it finishes the current one.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <stdint.h>
+
+#include "ptx_sm100.cuh"
 
 namespace h3q {
 
 constexpr int kRqMaxRows = 16;
 
 template <typename T>
-struct Raw;  // raw 16-byte words holding one lane's 16 input values
+struct Lane16;  // one lane's 16 values of a group: runs [8l, 8l+8) and [128+8l, 128+8l+8)
 
 template <>
-struct Raw<__nv_bfloat16> {
-  static constexpr int kWords = 2;
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, uint4 (&w)[kWords]) {
-    const uint4* s = reinterpret_cast<const uint4*>(p);
-    w[0] = __ldcs(s);
-    w[1] = __ldcs(s + 1);
-  }
-  // element 2i of a word is its low half, 2i+1 its high half
-  static __device__ __forceinline__ void unpack(const uint4 (&w)[kWords], float2 (&p)[8]) {
-    const uint32_t u[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
-    float v[16];
+struct Lane16<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* grp, int hl, float2 (&p)[8]) {
+    const uint4 a = *reinterpret_cast<const uint4*>(grp + 8 * hl);
+    const uint4 b = *reinterpret_cast<const uint4*>(grp + 128 + 8 * hl);
+    const uint32_t ua[4] = {a.x, a.y, a.z, a.w}, ub[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[2 * i] = __uint_as_float(u[i] << 16);
-      v[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+    for (int i = 0; i < 4; ++i) {  // element 2i of a word is its low half
+      p[2 * i] = make_float2(__uint_as_float(ua[i] << 16), __uint_as_float(ub[i] << 16));
+      p[2 * i + 1] = make_float2(__uint_as_float(ua[i] & 0xFFFF0000u), __uint_as_float(ub[i] & 0xFFFF0000u));
     }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) p[r] = make_float2(v[r], v[r + 8]);
   }
 };
 
 template <>
-struct Raw<float> {
-  static constexpr int kWords = 4;
-  static __device__ __forceinline__ void load(const float* p, uint4 (&w)[kWords]) {
-    const uint4* s = reinterpret_cast<const uint4*>(p);
-#pragma unroll
-    for (int i = 0; i < kWords; ++i) w[i] = __ldcs(s + i);
-  }
-  static __device__ __forceinline__ void unpack(const uint4 (&w)[kWords], float2 (&p)[8]) {
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[4 * i] = __uint_as_float(w[i].x);
-      v[4 * i + 1] = __uint_as_float(w[i].y);
-      v[4 * i + 2] = __uint_as_float(w[i].z);
-      v[4 * i + 3] = __uint_as_float(w[i].w);
-    }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) p[r] = make_float2(v[r], v[r + 8]);
+struct Lane16<float> {
+  static __device__ __forceinline__ void load(const float* grp, int hl, float2 (&p)[8]) {
+    const float4* a = reinterpret_cast<const float4*>(grp + 8 * hl);
+    const float4* b = reinterpret_cast<const float4*>(grp + 128 + 8 * hl);
+    const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
+    p[0] = make_float2(a0.x, b0.x); p[1] = make_float2(a0.y, b0.y);
+    p[2] = make_float2(a0.z, b0.z); p[3] = make_float2(a0.w, b0.w);
+    p[4] = make_float2(a1.x, b1.x); p[5] = make_float2(a1.y, b1.y);
+    p[6] = make_float2(a1.z, b1.z); p[7] = make_float2(a1.w, b1.w);
   }
 };
 
-// Unnormalized Walsh-Hadamard transform of one 256-group; p[r] = (v[r], v[r+8])
-// of lane hl's 16 elements 16 hl + r.
+// Unnormalized Walsh-Hadamard transform of one 256-group held by a half-warp.
 __device__ __forceinline__ void fwht256_halfwarp(float2 (&p)[8], int hl) {
   const float2 minus1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
-  for (int b = 0; b < 3; ++b) {  // index bits 0, 1, 2: pairs (r, r + 2^b) of packed registers
+  for (int b = 0; b < 3; ++b) {  // index bits 0, 1, 2: packed registers r and r + 2^b
     const int s = 1 << b;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
@@ -100,12 +89,7 @@ __device__ __forceinline__ void fwht256_halfwarp(float2 (&p)[8], int hl) {
     }
   }
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {  // index bit 3: inside each pair
-    const float lo = p[r].x, hi = p[r].y;
-    p[r] = make_float2(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
-  }
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {  // index bits 4-7 = lane bits 0-3 of the half-warp
+  for (int b = 0; b < 4; ++b) {  // index bits 3-6 = lane bits 0-3 of the half-warp
     const int m = 1 << b;
     const float sg = (hl & m) ? -1.0f : 1.0f;
     const float2 sign = make_float2(sg, sg);
@@ -113,10 +97,21 @@ __device__ __forceinline__ void fwht256_halfwarp(float2 (&p)[8], int hl) {
     for (int r = 0; r < 8; ++r) {
       const float2 other = make_float2(__shfl_xor_sync(0xFFFFFFFFu, p[r].x, m),
                                        __shfl_xor_sync(0xFFFFFFFFu, p[r].y, m));
-      // lower partner: own + other; upper partner: other - own
-      p[r] = __ffma2_rn(p[r], sign, other);
+      p[r] = __ffma2_rn(p[r], sign, other);  // lower lane: own + other; upper lane: other - own
     }
   }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {  // index bit 7: the two halves of each pair
+    const float lo = p[r].x, hi = p[r].y;
+    p[r] = make_float2(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
+  }
+}
+
+// max of three fp32 values (sm_100 three-input max).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -125,11 +120,12 @@ __device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t 
   return __byte_perm(ab, cd, 0x5410);
 }
 
-// Codes of one lane's 16 rotated values, as 4 words in natural element order.
-__device__ __forceinline__ uint4 quantize16(const float2 (&p)[8], float s16, float rs, bool exact_div) {
+// Codes of one lane's 16 rotated values: .x/.y = elements 8l..8l+7,
+// .z/.w = elements 128+8l .. 128+8l+7.
+__device__ __forceinline__ uint4 quantize16(const float2 (&p)[8], float s16, float rs) {
   const float2 magic = make_float2(12582912.0f, 12582912.0f);
   uint32_t ux[8], uy[8];
-  if (!exact_div) {
+  if (rs != 0.0f) {
     const float2 r2 = make_float2(rs, rs), ns2 = make_float2(-s16, -s16);
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
@@ -155,96 +151,153 @@ __device__ __forceinline__ uint4 quantize16(const float2 (&p)[8], float s16, flo
                     low_bytes4(uy[0], uy[1], uy[2], uy[3]), low_bytes4(uy[4], uy[5], uy[6], uy[7]));
 }
 
-// GPS = groups per half-warp slot and item. The host picks R rows per item and
-// W <= 32 / GPS warps so that R * G <= 2 * W * GPS.
-template <typename T, int GPS>
-__global__ void __launch_bounds__(1024 / GPS) rotquant_kernel(const T* __restrict__ x, int64_t M, int K, int R,
-                                                        int64_t items, int8_t* __restrict__ q,
-                                                        float* __restrict__ s_out) {
-  using L = Raw<T>;
-  __shared__ uint32_t row_amax[3][kRqMaxRows];
-  __shared__ float row_s16[kRqMaxRows], row_rs[kRqMaxRows];
-  const int hl = threadIdx.x & 15;
-  const int slot = threadIdx.x >> 4;
-  const int HW = blockDim.x >> 4;
-  const int G = K >> 8;
+struct RqArgs {
+  int64_t M;          // rows
+  int K;              // row length (multiple of 256)
+  int R;              // rows per work item
+  int64_t items;      // ceil(M / R)
+  int stages;         // shared-memory ring depth
+  uint32_t stage_bytes;
+  int8_t* q;
+  float* s_out;
+  uint64_t wait_limit_ns;
+};
 
+// Warp 0 is the producer; warps 1..W are consumers, W * 2 * GPS >= R * (K / 256).
+// MINB = 2 builds the kernel for blocks of at most 736 threads, two per SM.
+template <typename T, int GPS, int MINB>
+__global__ void __launch_bounds__(MINB == 2 ? 736 : 1024 / GPS + 32, MINB)
+    rotquant_kernel(const T* __restrict__ x, const RqArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(a.stages) * a.stage_bytes);
+  uint64_t* empty = full + a.stages;
+  uint32_t* row_amax = reinterpret_cast<uint32_t*>(empty + a.stages);  // [3][kRqMaxRows]
+  float* row_s16 = reinterpret_cast<float*>(row_amax + 3 * kRqMaxRows);
+  float* row_rs = row_s16 + kRqMaxRows;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(row_rs + kRqMaxRows);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_cons = blockDim.x - 32;
+  const int G = a.K >> 8;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], n_cons);
+    }
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (threadIdx.x < 3 * kRqMaxRows) row_amax[threadIdx.x] = 0u;
+  __syncthreads();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; item < a.items; item += gridDim.x) {
+        if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_limit_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int64_t row0 = item * a.R;
+        const int64_t nrows = (a.M - row0) < a.R ? (a.M - row0) : a.R;
+        const uint32_t bytes = static_cast<uint32_t>(nrows * a.K * int64_t(sizeof(T)));
+        mbar_arrive_expect_tx(&full[stage], bytes);
+        bulk_load(smem + size_t(stage) * a.stage_bytes, x + row0 * a.K, bytes, &full[stage], pol);
+        ++issued;
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {  // drain this block's own copies still in flight (bounded)
+        for (int s = 0; s < a.stages; ++s) {
+          if (issued <= s) continue;
+          const long last = ((issued - 1 - s) / a.stages) * a.stages + s;
+          mbar_wait_bounded(&full[s], static_cast<uint32_t>((last / a.stages) & 1), a.wait_limit_ns, nullptr);
+        }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int c = threadIdx.x - 32;
+  const int hl = c & 15;
+  const int slot = c >> 4;
+  const int HW = n_cons >> 4;
   int rr[GPS], gg[GPS];
   bool act[GPS];
 #pragma unroll
   for (int t = 0; t < GPS; ++t) {
     const int i = t * HW + slot;
-    act[t] = i < R * G;
+    act[t] = i < a.R * G;
     rr[t] = act[t] ? i / G : 0;
     gg[t] = act[t] ? i - rr[t] * G : 0;
   }
-  if (threadIdx.x < 3 * kRqMaxRows) (&row_amax[0][0])[threadIdx.x] = 0u;
-  __syncthreads();
 
-  auto load_item = [&](int64_t item, uint4 (&raw)[GPS][L::kWords]) {
-#pragma unroll
-    for (int t = 0; t < GPS; ++t) {
-      const int64_t row = item * R + rr[t];
-      if (act[t] && row < M) {
-        L::load(x + row * K + gg[t] * 256 + hl * 16, raw[t]);
-      } else {
-#pragma unroll
-        for (int w = 0; w < L::kWords; ++w) raw[t][w] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-  };
-
-  uint4 raw[GPS][L::kWords];
-  int64_t item = blockIdx.x;
-  if (item < items) load_item(item, raw);
-  for (int it = 0; item < items; item += gridDim.x, ++it) {
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int64_t item = blockIdx.x, it = 0; item < a.items; item += gridDim.x, ++it) {
+    mbar_wait_bounded(&full[stage], phase, a.wait_limit_ns, abort_flag);  // on expiry: garbage, no hang
+    const T* tile = reinterpret_cast<const T*>(smem + size_t(stage) * a.stage_bytes);
     float2 p[GPS][8];
 #pragma unroll
-    for (int t = 0; t < GPS; ++t) L::unpack(raw[t], p[t]);
-    const int64_t next = item + gridDim.x;
-    if (next < items) load_item(next, raw);  // in flight while this item is finished
-    const int buf = it % 3;
-    if (threadIdx.x < kRqMaxRows) row_amax[(it + 1) % 3][threadIdx.x] = 0u;
+    for (int t = 0; t < GPS; ++t) Lane16<T>::load(tile + rr[t] * a.K + gg[t] * 256, hl, p[t]);
+    mbar_arrive(&empty[stage]);  // this thread's reads of the stage are done
+    if (++stage == a.stages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+    const int buf = static_cast<int>(it % 3);
+    if (c < kRqMaxRows) row_amax[((it + 1) % 3) * kRqMaxRows + c] = 0u;
 
+    const int64_t row0 = item * a.R;
 #pragma unroll
     for (int t = 0; t < GPS; ++t) {
       fwht256_halfwarp(p[t], hl);
       float m = 0.0f;
 #pragma unroll
-      for (int r = 0; r < 8; ++r) m = fmaxf(m, fmaxf(fabsf(p[t][r].x), fabsf(p[t][r].y)));
+      for (int r = 0; r < 8; ++r) m = fmax3(m, fabsf(p[t][r].x), fabsf(p[t][r].y));
 #pragma unroll
       for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-      const int64_t row = item * R + rr[t];
-      if (hl == 0 && act[t] && row < M) atomicMax(&row_amax[buf][rr[t]], __float_as_uint(m));
+      if (hl == 0 && act[t] && row0 + rr[t] < a.M)
+        atomicMax(&row_amax[buf * kRqMaxRows + rr[t]], __float_as_uint(m));
     }
-    __syncthreads();
-    if (threadIdx.x < R) {
-      const int64_t row = item * R + threadIdx.x;
-      const float a = __uint_as_float(row_amax[buf][threadIdx.x]);
-      const float s16 = __fdiv_rn(a, 127.0f);
-      row_s16[threadIdx.x] = s16;
-      row_rs[threadIdx.x] = s16 >= 0x1p-100f ? __frcp_rn(s16) : 0.0f;
-      if (row < M) s_out[row] = __fmul_rn(s16, 0.0625f);
+    named_barrier(1, n_cons);
+    if (c < a.R) {
+      const float am = __uint_as_float(row_amax[buf * kRqMaxRows + c]);
+      const float s16 = __fdiv_rn(am, 127.0f);
+      row_s16[c] = s16;
+      row_rs[c] = s16 >= 0x1p-100f ? __frcp_rn(s16) : 0.0f;
+      if (row0 + c < a.M) a.s_out[row0 + c] = __fmul_rn(s16, 0.0625f);
     }
-    __syncthreads();
+    named_barrier(1, n_cons);
 #pragma unroll
     for (int t = 0; t < GPS; ++t) {
-      const int64_t row = item * R + rr[t];
-      const float s16 = row_s16[rr[t]];
-      const float rs = row_rs[rr[t]];
-      const uint4 codes = quantize16(p[t], s16, rs, rs == 0.0f);
-      if (act[t] && row < M)
-        *reinterpret_cast<uint4*>(q + row * K + gg[t] * 256 + hl * 16) = codes;
+      const int64_t row = row0 + rr[t];
+      const uint4 codes = quantize16(p[t], row_s16[rr[t]], row_rs[rr[t]]);
+      if (act[t] && row < a.M) {
+        int8_t* dst = a.q + row * a.K + gg[t] * 256 + 8 * hl;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(codes.x, codes.y);
+        *reinterpret_cast<uint2*>(dst + 128) = make_uint2(codes.z, codes.w);
+      }
     }
   }
 }
 
 struct RqShape {
-  int gps, warps, rows;
+  int gps, warps, rows;  // groups per half-warp slot, consumer warps, rows per item
 };
 
-// Rows per item, warps and groups per slot for a row of G groups: no idle slots
-// where possible, 256-1024 threads, fewest groups per slot.
+// Rows per item, consumer warps and groups per slot for a row of G groups: no
+// idle slots where possible, at least 256 consumer threads, fewest groups per
+// slot.
 inline RqShape rotquant_shape(int G) {
   RqShape best{0, 0, 0};
   double best_score = 1e30;
@@ -252,7 +305,8 @@ inline RqShape rotquant_shape(int G) {
     for (int R = 1; R <= kRqMaxRows; ++R) {
       const int slots = R * G;
       const int W = (slots + 2 * gps - 1) / (2 * gps);
-      if (W > 32 / gps) continue;  // the kernel is built for at most 1024 / gps threads
+      // consumers of a block built for 1024 / gps + 32 threads, at most 1024 with the producer
+      if (W > 32 / gps || W > 31) continue;
       const double waste = double(2 * W * gps - slots) / slots;
       const int threads = 32 * W;
       const double score = waste * 10.0 + (threads < 256 ? (256 - threads) / 256.0 : 0.0) + 0.05 * gps +
@@ -265,38 +319,65 @@ inline RqShape rotquant_shape(int G) {
   return best;
 }
 
-template <typename T, int GPS>
+inline size_t rotquant_smem_bytes(int stages, uint32_t stage_bytes) {
+  return size_t(stages) * stage_bytes + 2 * sizeof(uint64_t) * stages + (3 * kRqMaxRows + 2 * kRqMaxRows) * 4 +
+         16;
+}
+
+template <typename T, int GPS, int MINB>
 cudaError_t launch_rotquant_t(const T* x, int64_t rows, int64_t K, int8_t* q, float* s, const RqShape& sh,
-                              cudaStream_t stream) {
-  // blocks per SM for each block size, queried once (device 0 .. 15)
-  static int occ_cache[16][33] = {};
-  static int sm_cache[16] = {};
-  const int threads = 32 * sh.warps;
+                              uint64_t wait_limit_ns, cudaStream_t stream) {
+  RqArgs a;
+  a.M = rows;
+  a.K = static_cast<int>(K);
+  a.R = sh.rows;
+  a.items = (rows + sh.rows - 1) / sh.rows;
+  a.stage_bytes = static_cast<uint32_t>(int64_t(sh.rows) * K * int64_t(sizeof(T)));
+  // about 64 KB of loads in flight per block, 2 to 8 stages, under 110 KB so two blocks fit an SM
+  int stages = static_cast<int>((65536 + a.stage_bytes - 1) / a.stage_bytes);
+  stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
+  while (stages > 2 && rotquant_smem_bytes(stages, a.stage_bytes) > 110 * 1024) --stages;
+  a.stages = stages;
+  a.q = q;
+  a.s_out = s;
+  a.wait_limit_ns = wait_limit_ns;
+  const size_t smem = rotquant_smem_bytes(stages, a.stage_bytes);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  const int threads = 32 * (sh.warps + 1);
+
+  static int sm_count[16] = {};
+  static bool attr_set[16] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   dev &= 15;
-  if (sm_cache[dev] == 0) cudaDeviceGetAttribute(&sm_cache[dev], cudaDevAttrMultiProcessorCount, dev);
-  if (occ_cache[dev][sh.warps] == 0) {
-    int occ = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotquant_kernel<T, GPS>, threads, 0);
-    occ_cache[dev][sh.warps] = occ < 1 ? 1 : occ;
+  if (sm_count[dev] == 0) cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+  if (!attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(rotquant_kernel<T, GPS, MINB>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
   }
-  const int sms = sm_cache[dev], occ = occ_cache[dev][sh.warps];
-  const int64_t items = (rows + sh.rows - 1) / sh.rows;
-  const int64_t cap = int64_t(sms) * occ;
-  const unsigned grid = static_cast<unsigned>(items < cap ? items : cap);
-  rotquant_kernel<T, GPS><<<grid, threads, 0, stream>>>(x, rows, static_cast<int>(K), sh.rows, items, q, s);
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotquant_kernel<T, GPS, MINB>, threads, smem);
+  if (occ < 1) occ = 1;
+  const int64_t cap = int64_t(sm_count[dev]) * occ;
+  const unsigned grid = static_cast<unsigned>(a.items < cap ? a.items : cap);
+  rotquant_kernel<T, GPS, MINB><<<grid, threads, smem, stream>>>(x, a);
   return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t launch_rotquant(const T* x, int64_t rows, int64_t K, int8_t* q, float* s, cudaStream_t stream) {
+cudaError_t launch_rotquant(const T* x, int64_t rows, int64_t K, int8_t* q, float* s, uint64_t wait_limit_ns,
+                            cudaStream_t stream) {
   const RqShape sh = rotquant_shape(static_cast<int>(K / 256));
+  const bool two_per_sm = 32 * (sh.warps + 1) <= 736;
   switch (sh.gps) {
-    case 1: return launch_rotquant_t<T, 1>(x, rows, K, q, s, sh, stream);
-    case 2: return launch_rotquant_t<T, 2>(x, rows, K, q, s, sh, stream);
-    case 3: return launch_rotquant_t<T, 3>(x, rows, K, q, s, sh, stream);
-    default: return launch_rotquant_t<T, 4>(x, rows, K, q, s, sh, stream);
+    case 1:
+      return two_per_sm ? launch_rotquant_t<T, 1, 2>(x, rows, K, q, s, sh, wait_limit_ns, stream)
+                        : launch_rotquant_t<T, 1, 1>(x, rows, K, q, s, sh, wait_limit_ns, stream);
+    case 2: return launch_rotquant_t<T, 2, 1>(x, rows, K, q, s, sh, wait_limit_ns, stream);
+    case 3: return launch_rotquant_t<T, 3, 1>(x, rows, K, q, s, sh, wait_limit_ns, stream);
+    default: return launch_rotquant_t<T, 4, 1>(x, rows, K, q, s, sh, wait_limit_ns, stream);
   }
 }
 
