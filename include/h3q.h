@@ -112,6 +112,36 @@ h3q_status h3q_ffn(const void* x_bf16, int64_t M, int64_t K,
                    void* y_bf16, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * The FFN block of h3q_ffn, for callers that cannot allocate device memory.
+ * No passage of the pages corresponds to this call: it exists for the library's
+ * users. Some callers have no device allocator of their own (a host program
+ * that reaches this library only through plain pointers, or a plug-in whose
+ * device memory is owned entirely by the framework hosting it), and some must
+ * not allocate while serving, because cudaMalloc and cudaFree can synchronize
+ * the device and stall work on other streams. This call takes no workspace:
+ * its intermediates (xq, sx, h, hq, sh) live in one scratch array of
+ * H3Q_STATIC_SCRATCH_BYTES bytes that the library declares in device global
+ * memory. Every GPU that loads the library holds that array until the process
+ * exits. It allocates nothing and calls no allocating routine.
+ *   Arguments, layouts and results are those of h3q_ffn, minus the workspace.
+ *   Limit: h3q_ffn_workspace_size(M, K, F) <= H3Q_STATIC_SCRATCH_BYTES, else
+ *   H3Q_ERR_UNSUPPORTED and nothing is launched; for K = 5376, F = 14336 that
+ *   is M <= 1386 rows (the rows are independent, so a caller may split a
+ *   larger batch into chunks).
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the one array and it keeps the last call's contents:
+ *   calls that may overlap on the GPU (different streams without ordering
+ *   between them, or different host threads) race on it and must be
+ *   serialized by the caller.
+ */
+#define H3Q_STATIC_SCRATCH_BYTES (64u << 20)
+h3q_status h3q_ffn_static_scratch(const void* x_bf16, int64_t M, int64_t K,
+                                  const int8_t* w_gu, const float* s_gu, const void* b_gu, int64_t F,
+                                  const int8_t* w_down, const float* s_down, const void* b_down,
+                                  void* y_bf16, cudaStream_t stream);
+
+/*
  * Test hook: the same GEMM kernel with the raw int32 accumulators as output.
  *   xq [M, K], wq [N, K] int8; acc [M, N] int32. K % 128 == 0, N % 8 == 0.
  */

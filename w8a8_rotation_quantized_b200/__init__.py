@@ -33,6 +33,7 @@ _SIGS = {
     "h3q_linear_w8a8": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _INT, _P, _P]),
     "h3q_ffn_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "h3q_ffn": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]),
+    "h3q_ffn_static_scratch": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _P, _P]),
     "h3q_gemm_s32": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P]),
     "h3q_get_device_status": (_INT, [_P]),
     "h3q_set_wait_limit_ns": (None, [_U64]),
@@ -104,6 +105,20 @@ def h3q_ffn(x, w_gu, s_gu, w_down, s_down, y, workspace, b_gu=None, b_down=None,
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib.h3q_ffn(_ptr(x), M, K, _ptr(w_gu), _ptr(s_gu), _ptr(b_gu), F, _ptr(w_down), _ptr(s_down),
                        _ptr(b_down), _ptr(y), _ptr(workspace), nbytes, _stream(stream)), "h3q_ffn")
+
+
+H3Q_STATIC_SCRATCH_BYTES = 64 << 20
+
+
+def h3q_ffn_static_scratch(x, w_gu, s_gu, w_down, s_down, y, b_gu=None, b_down=None, stream=None) -> None:
+    """h3q_ffn without a workspace, for callers that cannot allocate device memory:
+    the intermediates live in the library's fixed 64 MiB device array, shared by
+    all calls (calls that may overlap on the GPU must be serialized)."""
+    M, K = x.shape
+    F = w_gu.shape[0] // 2
+    _check(lib.h3q_ffn_static_scratch(_ptr(x), M, K, _ptr(w_gu), _ptr(s_gu), _ptr(b_gu), F, _ptr(w_down),
+                                      _ptr(s_down), _ptr(b_down), _ptr(y), _stream(stream)),
+           "h3q_ffn_static_scratch")
 
 
 def h3q_gemm_s32(xq, wq, acc, stream=None) -> None:

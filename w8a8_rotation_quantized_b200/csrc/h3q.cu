@@ -114,6 +114,24 @@ FfnLayout ffn_layout(int64_t M, int64_t K, int64_t F) {
   return l;
 }
 
+// Scratch for h3q_ffn_static_scratch: a fixed device array, so that call needs
+// no allocation. In host code this name only stands for the array; its device
+// address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_static_scratch[H3Q_STATIC_SCRATCH_BYTES];
+
+void* static_scratch_address(int device) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  if (device < 0 || device >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[device] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+    addr[device] = p;
+  }
+  return addr[device];
+}
+
 }  // namespace
 
 extern "C" {
@@ -210,6 +228,20 @@ h3q_status h3q_ffn(const void* x_bf16, int64_t M, int64_t K, const int8_t* w_gu,
   st = h3q_rotate_quant(h, M, F, hq, sh, stream);
   if (st != H3Q_OK) return st;
   return h3q_linear_w8a8(hq, sh, M, F, w_down, s_down, K, b_down, H3Q_EPI_NONE, y_bf16, stream);
+}
+
+h3q_status h3q_ffn_static_scratch(const void* x_bf16, int64_t M, int64_t K, const int8_t* w_gu, const float* s_gu,
+                                  const void* b_gu, int64_t F, const int8_t* w_down, const float* s_down,
+                                  const void* b_down, void* y_bf16, cudaStream_t stream) {
+  if (M < 0 || !valid_k(K) || !valid_k(F)) return H3Q_ERR_INVALID_ARG;
+  if (M == 0) return H3Q_OK;
+  if (ffn_layout(M, K, F).total > size_t(H3Q_STATIC_SCRATCH_BYTES)) return H3Q_ERR_UNSUPPORTED;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return H3Q_ERR_CUDA;
+  void* scratch = static_scratch_address(device);
+  if (scratch == nullptr) return H3Q_ERR_CUDA;
+  return h3q_ffn(x_bf16, M, K, w_gu, s_gu, b_gu, F, w_down, s_down, b_down, y_bf16, scratch,
+                 size_t(H3Q_STATIC_SCRATCH_BYTES), stream);
 }
 
 h3q_status h3q_get_device_status(cudaStream_t stream) {
