@@ -59,6 +59,8 @@ def test_rotate_quant_bitexact(h3q, cuda_device, M, K):
         x_h[5] = 0
         x_h[5, K // 2] = 0x3F80          # a single 1.0: flat rotated group
         x_h[6] = 0xC2C8                  # constant -100 row
+        # tiny row (|x| ~ 2^-109): its scale is below 2^-100
+        x_h[4] = (0x0900 | (x_h[4] & 0x807F)).astype(np.uint16)
     x = to_dev(x_h, cuda_device)
     xq = torch.empty((M, K), dtype=torch.int8, device=cuda_device)
     sx = torch.empty(M, dtype=torch.float32, device=cuda_device)

@@ -6,32 +6,35 @@
 // work items (R whole rows, contiguous in memory) into a ring of shared-memory
 // stages with 1D bulk copies (cp.async.bulk, completion on an mbarrier), so
 // several items are in flight per block while the consumer warps work. Each row
-// is read from HBM once and its codes written once.
+// is read from HBM once and its codes are written once.
 //
-// Work split: a half-warp (16 lanes) of the consumers owns one 256-group of a
-// row. Lane l of the half reads two 16-byte runs of the group from shared
-// memory: elements 8l .. 8l+7 and 128+8l .. 128+8l+7 (bank-conflict free), kept
-// as packed pairs p[r] = (v[r], v[r+8]) of element 8l+r and 128+8l+r. Index bits
-// 0-2 are register bits, bits 3-6 the lane bits, bit 7 the pair half.
-//
-// Rotation: the unnormalized Walsh-Hadamard butterflies in ascending index-bit
-// order: bits 0-2 on packed pairs with the sm_100 two-wide fp32 add, bits 3-6
-// across lanes by shuffles (a fused multiply by +-1 and add, one rounding),
-// bit 7 inside each pair. Every butterfly is one correctly rounded fp32 add or
-// subtract, so each rotated value has the same bits as the pairwise-tree sum of
-// the explicit H/16 product. The 1/16 moves to the scale: y16 = 16 y and
-// s16 = max|y16| / 127 = 16 s exactly, and y16 / s16 = y / s, so the codes are
-// unchanged.
+// Rotation of one 256-group by a half-warp (16 lanes), seen as a 16 x 16 matrix
+// X[a][b] = x[16a + b]:
+//   phase A  lane a holds row a (16 contiguous elements) and applies the
+//            butterflies of index bits 0-3 in registers;
+//   transpose through a per-half-warp shared-memory scratch (fp32, chunks
+//            swizzled so both the row writes and the column reads are free of
+//            bank conflicts);
+//   phase B  lane b holds column b and applies the butterflies of bits 4-7.
+// Each phase keeps its 16 values as packed pairs (v[r], v[r+8]) and runs three
+// stages on the sm_100 two-wide fp32 add and the fourth inside each pair. The
+// bits are processed in ascending order and every butterfly is one correctly
+// rounded fp32 add or subtract, so each rotated value has the same bits as the
+// pairwise-tree sum of the explicit H/16 product. No shuffle is needed. The
+// 1/16 moves to the scale: y16 = 16 y and s16 = max|y16| / 127 = 16 s exactly,
+// and y16 / s16 = y / s, so the codes are unchanged.
 //
 // Quantization needs rne(RN(y / s)) per element. Each row gets rs = RN(1/s)
 // once; each quotient is q0 = RN(y rs) refined twice with exact FMA residuals,
 // e = y - q s, q <- RN(q + e rs) (Markstein, "Computation of elementary
 // functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
 // 1990): after the first step q is within one ulp of y/s, and the second step
-// returns the correctly rounded quotient. Rows whose scale is below 2^-100
-// (never met in practice) use IEEE division. The integer is read from the bits
+// returns the correctly rounded quotient. Rows whose scale is below 2^-100 are
+// first rescaled by 2^64 (exact). The integer is read from the bits
 // of q + 1.5*2^23, whose add rounds half to even; its low byte is the int8 code.
-// |y| <= max|y| bounds y/s by 127 (1 + 2^-23), so no clamp is needed.
+// |y| <= max|y| bounds y/s by 127 (1 + 2^-23), so no clamp is needed. The codes
+// of a column are scattered bytes of the group; they pass through the slot's
+// shared buffer and leave as one 16-byte store per lane.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -42,42 +45,43 @@
 namespace h3q {
 
 constexpr int kRqMaxRows = 16;
+constexpr int kRqSlotBytes = 1024 + 64;  // per half-warp: 16 x 16 fp32 scratch + 64 B so slots shift banks by 16
 
 template <typename T>
-struct Lane16;  // one lane's 16 values of a group: runs [8l, 8l+8) and [128+8l, 128+8l+8)
+struct Row16;  // lane a's 16 contiguous elements 16a .. 16a+15 of a group, as pairs (v[r], v[r+8])
 
 template <>
-struct Lane16<__nv_bfloat16> {
-  static __device__ __forceinline__ void load(const __nv_bfloat16* grp, int hl, float2 (&p)[8]) {
-    const uint4 a = *reinterpret_cast<const uint4*>(grp + 8 * hl);
-    const uint4 b = *reinterpret_cast<const uint4*>(grp + 128 + 8 * hl);
-    const uint32_t ua[4] = {a.x, a.y, a.z, a.w}, ub[4] = {b.x, b.y, b.z, b.w};
+struct Row16<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* grp, int a, float2 (&p)[8]) {
+    const uint4* row = reinterpret_cast<const uint4*>(grp + 16 * a);
+    const uint4 lo = row[0], hi = row[1];  // elements 0-7 and 8-15
+    const uint32_t ul[4] = {lo.x, lo.y, lo.z, lo.w}, uh[4] = {hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {  // element 2i of a word is its low half
-      p[2 * i] = make_float2(__uint_as_float(ua[i] << 16), __uint_as_float(ub[i] << 16));
-      p[2 * i + 1] = make_float2(__uint_as_float(ua[i] & 0xFFFF0000u), __uint_as_float(ub[i] & 0xFFFF0000u));
+      p[2 * i] = make_float2(__uint_as_float(ul[i] << 16), __uint_as_float(uh[i] << 16));
+      p[2 * i + 1] = make_float2(__uint_as_float(ul[i] & 0xFFFF0000u), __uint_as_float(uh[i] & 0xFFFF0000u));
     }
   }
 };
 
 template <>
-struct Lane16<float> {
-  static __device__ __forceinline__ void load(const float* grp, int hl, float2 (&p)[8]) {
-    const float4* a = reinterpret_cast<const float4*>(grp + 8 * hl);
-    const float4* b = reinterpret_cast<const float4*>(grp + 128 + 8 * hl);
-    const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
-    p[0] = make_float2(a0.x, b0.x); p[1] = make_float2(a0.y, b0.y);
-    p[2] = make_float2(a0.z, b0.z); p[3] = make_float2(a0.w, b0.w);
-    p[4] = make_float2(a1.x, b1.x); p[5] = make_float2(a1.y, b1.y);
-    p[6] = make_float2(a1.z, b1.z); p[7] = make_float2(a1.w, b1.w);
+struct Row16<float> {
+  static __device__ __forceinline__ void load(const float* grp, int a, float2 (&p)[8]) {
+    const float4* row = reinterpret_cast<const float4*>(grp + 16 * a);
+    const float4 c0 = row[0], c1 = row[1], c2 = row[2], c3 = row[3];
+    p[0] = make_float2(c0.x, c2.x); p[1] = make_float2(c0.y, c2.y);
+    p[2] = make_float2(c0.z, c2.z); p[3] = make_float2(c0.w, c2.w);
+    p[4] = make_float2(c1.x, c3.x); p[5] = make_float2(c1.y, c3.y);
+    p[6] = make_float2(c1.z, c3.z); p[7] = make_float2(c1.w, c3.w);
   }
 };
 
-// Unnormalized Walsh-Hadamard transform of one 256-group held by a half-warp.
-__device__ __forceinline__ void fwht256_halfwarp(float2 (&p)[8], int hl) {
+// Unnormalized 16-point Walsh-Hadamard transform of v[0..15] held as
+// p[r] = (v[r], v[r+8]): bits 0-2 on packed pairs, then bit 3 inside each pair.
+__device__ __forceinline__ void fwht16(float2 (&p)[8]) {
   const float2 minus1 = make_float2(-1.0f, -1.0f);
 #pragma unroll
-  for (int b = 0; b < 3; ++b) {  // index bits 0, 1, 2: packed registers r and r + 2^b
+  for (int b = 0; b < 3; ++b) {
     const int s = 1 << b;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
@@ -89,22 +93,41 @@ __device__ __forceinline__ void fwht256_halfwarp(float2 (&p)[8], int hl) {
     }
   }
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {  // index bits 3-6 = lane bits 0-3 of the half-warp
-    const int m = 1 << b;
-    const float sg = (hl & m) ? -1.0f : 1.0f;
-    const float2 sign = make_float2(sg, sg);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const float2 other = make_float2(__shfl_xor_sync(0xFFFFFFFFu, p[r].x, m),
-                                       __shfl_xor_sync(0xFFFFFFFFu, p[r].y, m));
-      p[r] = __ffma2_rn(p[r], sign, other);  // lower lane: own + other; upper lane: other - own
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {  // index bit 7: the two halves of each pair
+  for (int r = 0; r < 8; ++r) {
     const float lo = p[r].x, hi = p[r].y;
     p[r] = make_float2(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
   }
+}
+
+// Scratch layout: row a holds 16 fp32 values; its 16-byte chunk k sits at chunk
+// position k ^ ((a >> 1) & 3) of the row.
+// Rotates one group: on return, p[r] = (y16[16 r + b], y16[16 (r + 8) + b]) for
+// this lane's column b = hl. `scratch` is the half-warp's private fp32 area.
+template <typename T>
+__device__ __forceinline__ void rotate_group(const T* grp, int hl, float* scratch, float2 (&p)[8]) {
+  Row16<T>::load(grp, hl, p);
+  fwht16(p);  // index bits 0-3
+  const int sw = (hl >> 1) & 3;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {  // row hl, chunk k = elements 4k .. 4k+3
+    const float4 c = k < 2 ? make_float4(p[4 * k].x, p[4 * k + 1].x, p[4 * k + 2].x, p[4 * k + 3].x)
+                           : make_float4(p[4 * k - 8].y, p[4 * k - 7].y, p[4 * k - 6].y, p[4 * k - 5].y);
+    *reinterpret_cast<float4*>(scratch + 16 * hl + 4 * (k ^ sw)) = c;
+  }
+  __syncwarp();
+  // column hl: row r's element sits at 16 r + 4 ((hl >> 2) ^ (r >> 1) & 3) + (hl & 3);
+  // four base pointers (one per value of r >> 1 & 3) leave an immediate offset per row
+  const float* col = scratch + (hl & 3);
+  const int x = hl >> 2;
+  const float* b0 = col + 4 * (x & 3);
+  const float* b1 = col + 4 * ((x ^ 1) & 3);
+  const float* b2 = col + 4 * ((x ^ 2) & 3);
+  const float* b3 = col + 4 * ((x ^ 3) & 3);
+  const float* base[4] = {b0, b1, b2, b3};
+#pragma unroll
+  for (int r = 0; r < 8; ++r) p[r] = make_float2(base[(r >> 1) & 3][16 * r], base[((r + 8) >> 1) & 3][16 * (r + 8)]);
+  __syncwarp();  // the scratch is rewritten next (codes or the next group)
+  fwht16(p);     // index bits 4-7
 }
 
 // max of three fp32 values (sm_100 three-input max).
@@ -114,41 +137,40 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-__device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  const uint32_t ab = __byte_perm(a, b, 0x0040);  // [a.b0, b.b0, -, -]
-  const uint32_t cd = __byte_perm(c, d, 0x0040);
-  return __byte_perm(ab, cd, 0x5410);
+// Per-row quotient constants: y / s is formed as (y f) / (s f) with f = 2^64 for
+// rows whose scale is below 2^-100 (an exact rescaling that keeps 1 / (s f) in
+// range), f = 1 otherwise; rs = RN(1 / (s f)), and rs = 0 for an all-zero row
+// (whose codes are then 0).
+struct RowQuot {
+  float f, sf, rs;
+};
+
+__device__ __forceinline__ RowQuot row_quotient(float s16) {
+  RowQuot r;
+  r.f = s16 < 0x1p-100f ? 0x1p64f : 1.0f;
+  r.sf = __fmul_rn(s16, r.f);
+  r.rs = s16 != 0.0f ? __frcp_rn(r.sf) : 0.0f;
+  return r;
 }
 
-// Codes of one lane's 16 rotated values: .x/.y = elements 8l..8l+7,
-// .z/.w = elements 128+8l .. 128+8l+7.
-__device__ __forceinline__ uint4 quantize16(const float2 (&p)[8], float s16, float rs) {
+// int8 codes rne(y16 / s16) of this lane's column hl, written as bytes into the
+// group's 256-byte code buffer at element positions 16 r + hl and 16 (r + 8) + hl.
+__device__ __forceinline__ void quantize_column(const float2 (&p)[8], const RowQuot& rq, int hl,
+                                                uint8_t* codes) {
   const float2 magic = make_float2(12582912.0f, 12582912.0f);
-  uint32_t ux[8], uy[8];
-  if (rs != 0.0f) {
-    const float2 r2 = make_float2(rs, rs), ns2 = make_float2(-s16, -s16);
+  const float2 f2 = make_float2(rq.f, rq.f), r2 = make_float2(rq.rs, rq.rs), ns2 = make_float2(-rq.sf, -rq.sf);
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      float2 q = __fmul2_rn(p[r], r2);
-      float2 e = __ffma2_rn(q, ns2, p[r]);
-      q = __ffma2_rn(e, r2, q);
-      e = __ffma2_rn(q, ns2, p[r]);
-      q = __ffma2_rn(e, r2, q);
-      const float2 u = __fadd2_rn(q, magic);
-      ux[r] = __float_as_uint(u.x);
-      uy[r] = __float_as_uint(u.y);
-    }
-  } else {
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const float qx = s16 != 0.0f ? __fdiv_rn(p[r].x, s16) : 0.0f;
-      const float qy = s16 != 0.0f ? __fdiv_rn(p[r].y, s16) : 0.0f;
-      ux[r] = __float_as_uint(__fadd_rn(qx, 12582912.0f));
-      uy[r] = __float_as_uint(__fadd_rn(qy, 12582912.0f));
-    }
+  for (int r = 0; r < 8; ++r) {
+    const float2 y = __fmul2_rn(p[r], f2);  // exact
+    float2 q = __fmul2_rn(y, r2);
+    float2 e = __ffma2_rn(q, ns2, y);
+    q = __ffma2_rn(e, r2, q);
+    e = __ffma2_rn(q, ns2, y);
+    q = __ffma2_rn(e, r2, q);
+    const float2 u = __fadd2_rn(q, magic);
+    codes[16 * r + hl] = static_cast<uint8_t>(__float_as_uint(u.x));
+    codes[16 * (r + 8) + hl] = static_cast<uint8_t>(__float_as_uint(u.y));
   }
-  return make_uint4(low_bytes4(ux[0], ux[1], ux[2], ux[3]), low_bytes4(ux[4], ux[5], ux[6], ux[7]),
-                    low_bytes4(uy[0], uy[1], uy[2], uy[3]), low_bytes4(uy[4], uy[5], uy[6], uy[7]));
 }
 
 struct RqArgs {
@@ -163,21 +185,33 @@ struct RqArgs {
   uint64_t wait_limit_ns;
 };
 
-// Warp 0 is the producer; warps 1..W are consumers, W * 2 * GPS >= R * (K / 256).
-// MINB = 2 builds the kernel for blocks of at most 736 threads, two per SM.
-template <typename T, int GPS, int MINB>
-__global__ void __launch_bounds__(MINB == 2 ? 736 : 1024 / GPS + 32, MINB)
+struct RqShape {
+  int gps, warps, rows, stages;  // groups per half-warp slot, consumer warps, rows per item, ring depth
+  bool small;                    // built for three blocks per SM
+};
+
+inline size_t rotquant_smem_bytes(int stages, uint32_t stage_bytes, int warps) {
+  return size_t(stages) * stage_bytes + size_t(2 * warps) * kRqSlotBytes + 2 * sizeof(uint64_t) * stages +
+         3 * kRqMaxRows * 4 + 16;
+}
+
+// Warp 0 is the producer; warps 1..W are consumers with 2W half-warp slots, each
+// taking GPS groups per item: 2 * W * GPS >= R * (K / 256). SMALL builds for
+// blocks of at most 16 warps, three per SM (40 registers); otherwise up to 32
+// warps, one per SM.
+template <typename T, int GPS, bool SMALL>
+__global__ void __launch_bounds__(SMALL ? 512 : 1024, SMALL ? 3 : 1)
     rotquant_kernel(const T* __restrict__ x, const RqArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(a.stages) * a.stage_bytes);
+  const int n_cons = blockDim.x - 32;
+  const int HW = n_cons >> 4;
+  uint8_t* scratch_base = smem + size_t(a.stages) * a.stage_bytes;  // HW slots of kRqSlotBytes
+  uint64_t* full = reinterpret_cast<uint64_t*>(scratch_base + size_t(HW) * kRqSlotBytes);
   uint64_t* empty = full + a.stages;
   uint32_t* row_amax = reinterpret_cast<uint32_t*>(empty + a.stages);  // [3][kRqMaxRows]
-  float* row_s16 = reinterpret_cast<float*>(row_amax + 3 * kRqMaxRows);
-  float* row_rs = row_s16 + kRqMaxRows;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(row_rs + kRqMaxRows);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(row_amax + 3 * kRqMaxRows);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_cons = blockDim.x - 32;
   const int G = a.K >> 8;
 
   if (threadIdx.x == 0) {
@@ -230,7 +264,8 @@ __global__ void __launch_bounds__(MINB == 2 ? 736 : 1024 / GPS + 32, MINB)
   const int c = threadIdx.x - 32;
   const int hl = c & 15;
   const int slot = c >> 4;
-  const int HW = n_cons >> 4;
+  float* scratch = reinterpret_cast<float*>(scratch_base + size_t(slot) * kRqSlotBytes);
+  uint8_t* codes_buf = reinterpret_cast<uint8_t*>(scratch);  // reused once the group is rotated
   int rr[GPS], gg[GPS];
   bool act[GPS];
 #pragma unroll
@@ -241,26 +276,22 @@ __global__ void __launch_bounds__(MINB == 2 ? 736 : 1024 / GPS + 32, MINB)
     gg[t] = act[t] ? i - rr[t] * G : 0;
   }
 
+  // Row slot buffers of the absmax: item k uses buffer k % 3; buffer (k + 1) % 3,
+  // last read before barrier k - 1, is cleared before barrier k, ahead of item
+  // k + 1's atomics.
   int stage = 0;
   uint32_t phase = 0;
   for (int64_t item = blockIdx.x, it = 0; item < a.items; item += gridDim.x, ++it) {
     mbar_wait_bounded(&full[stage], phase, a.wait_limit_ns, abort_flag);  // on expiry: garbage, no hang
     const T* tile = reinterpret_cast<const T*>(smem + size_t(stage) * a.stage_bytes);
-    float2 p[GPS][8];
-#pragma unroll
-    for (int t = 0; t < GPS; ++t) Lane16<T>::load(tile + rr[t] * a.K + gg[t] * 256, hl, p[t]);
-    mbar_arrive(&empty[stage]);  // this thread's reads of the stage are done
-    if (++stage == a.stages) {
-      stage = 0;
-      phase ^= 1u;
-    }
     const int buf = static_cast<int>(it % 3);
     if (c < kRqMaxRows) row_amax[((it + 1) % 3) * kRqMaxRows + c] = 0u;
-
     const int64_t row0 = item * a.R;
+
+    float2 p[GPS][8];
 #pragma unroll
     for (int t = 0; t < GPS; ++t) {
-      fwht256_halfwarp(p[t], hl);
+      rotate_group(tile + rr[t] * a.K + gg[t] * 256, hl, scratch, p[t]);
       float m = 0.0f;
 #pragma unroll
       for (int r = 0; r < 8; ++r) m = fmax3(m, fabsf(p[t][r].x), fabsf(p[t][r].y));
@@ -269,116 +300,142 @@ __global__ void __launch_bounds__(MINB == 2 ? 736 : 1024 / GPS + 32, MINB)
       if (hl == 0 && act[t] && row0 + rr[t] < a.M)
         atomicMax(&row_amax[buf * kRqMaxRows + rr[t]], __float_as_uint(m));
     }
-    named_barrier(1, n_cons);
-    if (c < a.R) {
-      const float am = __uint_as_float(row_amax[buf * kRqMaxRows + c]);
-      const float s16 = __fdiv_rn(am, 127.0f);
-      row_s16[c] = s16;
-      row_rs[c] = s16 >= 0x1p-100f ? __frcp_rn(s16) : 0.0f;
-      if (row0 + c < a.M) a.s_out[row0 + c] = __fmul_rn(s16, 0.0625f);
+    mbar_arrive(&empty[stage]);  // this thread's reads of the stage are done
+    if (++stage == a.stages) {
+      stage = 0;
+      phase ^= 1u;
     }
     named_barrier(1, n_cons);
 #pragma unroll
     for (int t = 0; t < GPS; ++t) {
       const int64_t row = row0 + rr[t];
-      const uint4 codes = quantize16(p[t], row_s16[rr[t]], row_rs[rr[t]]);
-      if (act[t] && row < a.M) {
-        int8_t* dst = a.q + row * a.K + gg[t] * 256 + 8 * hl;
-        *reinterpret_cast<uint2*>(dst) = make_uint2(codes.x, codes.y);
-        *reinterpret_cast<uint2*>(dst + 128) = make_uint2(codes.z, codes.w);
-      }
+      const float am = __uint_as_float(row_amax[buf * kRqMaxRows + rr[t]]);
+      const float s16 = __fdiv_rn(am, 127.0f);
+      if (hl == 0 && gg[t] == 0 && act[t] && row < a.M) a.s_out[row] = __fmul_rn(s16, 0.0625f);
+      quantize_column(p[t], row_quotient(s16), hl, codes_buf);
+      __syncwarp();
+      const uint4 out = *reinterpret_cast<const uint4*>(codes_buf + 16 * hl);  // elements 16 hl .. 16 hl + 15
+      __syncwarp();  // before the buffer is reused
+      if (act[t] && row < a.M) *reinterpret_cast<uint4*>(a.q + row * a.K + gg[t] * 256 + 16 * hl) = out;
     }
   }
 }
 
-struct RqShape {
-  int gps, warps, rows;  // groups per half-warp slot, consumer warps, rows per item
-};
+// ----------------------------------------------------------------------------
+// Host side: shape choice and launch.
 
-// Rows per item, consumer warps and groups per slot for a row of G groups: no
-// idle slots where possible, at least 256 consumer threads, fewest groups per
-// slot.
-inline RqShape rotquant_shape(int G) {
-  RqShape best{0, 0, 0};
-  double best_score = 1e30;
-  for (int gps = 1; gps <= 4; ++gps)
-    for (int R = 1; R <= kRqMaxRows; ++R) {
-      const int slots = R * G;
-      const int W = (slots + 2 * gps - 1) / (2 * gps);
-      // consumers of a block built for 1024 / gps + 32 threads, at most 1024 with the producer
-      if (W > 32 / gps || W > 31) continue;
-      const double waste = double(2 * W * gps - slots) / slots;
-      const int threads = 32 * W;
-      const double score = waste * 10.0 + (threads < 256 ? (256 - threads) / 256.0 : 0.0) + 0.05 * gps +
-                           0.001 * R;
-      if (score < best_score) {
-        best_score = score;
-        best = {gps, W, R};
+template <typename T, int GPS, bool SMALL>
+cudaError_t rotquant_prepare_attr(int dev) {
+  static bool done[16] = {};
+  if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
+  if (done[dev]) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(rotquant_kernel<T, GPS, SMALL>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
+
+template <typename T, int GPS, bool SMALL>
+int rotquant_occupancy_t(int threads, size_t smem, int dev) {
+  if (rotquant_prepare_attr<T, GPS, SMALL>(dev) != cudaSuccess) return 0;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotquant_kernel<T, GPS, SMALL>, threads, smem) !=
+      cudaSuccess)
+    return 0;
+  return occ;
+}
+
+template <typename T>
+int rotquant_occupancy(int gps, bool small, int threads, size_t smem, int dev) {
+  if (gps == 1) return small ? rotquant_occupancy_t<T, 1, true>(threads, smem, dev)
+                             : rotquant_occupancy_t<T, 1, false>(threads, smem, dev);
+  return small ? rotquant_occupancy_t<T, 2, true>(threads, smem, dev)
+               : rotquant_occupancy_t<T, 2, false>(threads, smem, dev);
+}
+
+// For a row of G groups: among shapes with 1 or 2 groups per slot, up to 8 rows
+// per item and 2 to 6 stages, keep the one with the most consumer warps doing
+// useful work per SM (occupancy times the share of busy slots), then the most
+// loads in flight per SM (up to 128 KB).
+template <typename T>
+RqShape rotquant_plan(int K, int dev, int* blocks_per_sm) {
+  static RqShape cache[16][65] = {};
+  static int cache_occ[16][65] = {};
+  const int G = K / 256;
+  if (dev >= 0 && dev < 16 && G <= 64 && cache[dev][G].gps != 0) {
+    *blocks_per_sm = cache_occ[dev][G];
+    return cache[dev][G];
+  }
+  RqShape best{0, 0, 0, 0, false};
+  int best_occ = 0;
+  double best_score = -1.0;
+  for (int gps = 1; gps <= 2; ++gps)
+    for (int R = 1; R <= 8 && R <= kRqMaxRows; ++R)
+      for (int small = 1; small >= 0; --small) {
+        const int slots = R * G;
+        const int W = (slots + 2 * gps - 1) / (2 * gps);
+        const int threads = 32 * (W + 1);
+        if (threads > (small ? 512 : 1024)) continue;
+        const uint32_t stage_bytes = static_cast<uint32_t>(int64_t(R) * K * int64_t(sizeof(T)));
+        for (int stages = 2; stages <= 6; ++stages) {
+          const size_t smem = rotquant_smem_bytes(stages, stage_bytes, W);
+          if (smem > 227 * 1024) break;
+          const int occ = rotquant_occupancy<T>(gps, small != 0, threads, smem, dev);
+          if (occ < 1) break;
+          // useful consumer warps per SM, then loads in flight per SM (capped)
+          const double busy = double(slots) / double(2 * W * gps);
+          const double inflight = double(occ) * stages * stage_bytes;
+          const double score = occ * W * busy + 4.0 * (inflight < 131072.0 ? inflight : 131072.0) / 131072.0 -
+                               0.01 * gps - 0.001 * R;
+          if (score > best_score) {
+            best_score = score;
+            best = {gps, W, R, stages, small != 0};
+            best_occ = occ;
+          }
+        }
       }
-    }
+  if (dev >= 0 && dev < 16 && G <= 64 && best.gps != 0) {
+    cache[dev][G] = best;
+    cache_occ[dev][G] = best_occ;
+  }
+  *blocks_per_sm = best_occ;
   return best;
 }
 
-inline size_t rotquant_smem_bytes(int stages, uint32_t stage_bytes) {
-  return size_t(stages) * stage_bytes + 2 * sizeof(uint64_t) * stages + (3 * kRqMaxRows + 2 * kRqMaxRows) * 4 +
-         16;
-}
-
-template <typename T, int GPS, int MINB>
-cudaError_t launch_rotquant_t(const T* x, int64_t rows, int64_t K, int8_t* q, float* s, const RqShape& sh,
-                              uint64_t wait_limit_ns, cudaStream_t stream) {
+template <typename T>
+cudaError_t launch_rotquant(const T* x, int64_t rows, int64_t K, int8_t* q, float* s, uint64_t wait_limit_ns,
+                            cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static int sm_count[16] = {};
+  if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
+  if (sm_count[dev] == 0) cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+  int occ = 0;
+  const RqShape sh = rotquant_plan<T>(static_cast<int>(K), dev, &occ);
+  if (sh.gps == 0) return cudaErrorInvalidConfiguration;
   RqArgs a;
   a.M = rows;
   a.K = static_cast<int>(K);
   a.R = sh.rows;
   a.items = (rows + sh.rows - 1) / sh.rows;
   a.stage_bytes = static_cast<uint32_t>(int64_t(sh.rows) * K * int64_t(sizeof(T)));
-  // about 64 KB of loads in flight per block, 2 to 8 stages, under 110 KB so two blocks fit an SM
-  int stages = static_cast<int>((65536 + a.stage_bytes - 1) / a.stage_bytes);
-  stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
-  while (stages > 2 && rotquant_smem_bytes(stages, a.stage_bytes) > 110 * 1024) --stages;
-  a.stages = stages;
+  a.stages = sh.stages;
   a.q = q;
   a.s_out = s;
   a.wait_limit_ns = wait_limit_ns;
-  const size_t smem = rotquant_smem_bytes(stages, a.stage_bytes);
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  const size_t smem = rotquant_smem_bytes(sh.stages, a.stage_bytes, sh.warps);
   const int threads = 32 * (sh.warps + 1);
-
-  static int sm_count[16] = {};
-  static bool attr_set[16] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  dev &= 15;
-  if (sm_count[dev] == 0) cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
-  if (!attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(rotquant_kernel<T, GPS, MINB>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
-  int occ = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotquant_kernel<T, GPS, MINB>, threads, smem);
-  if (occ < 1) occ = 1;
   const int64_t cap = int64_t(sm_count[dev]) * occ;
   const unsigned grid = static_cast<unsigned>(a.items < cap ? a.items : cap);
-  rotquant_kernel<T, GPS, MINB><<<grid, threads, smem, stream>>>(x, a);
-  return cudaGetLastError();
-}
-
-template <typename T>
-cudaError_t launch_rotquant(const T* x, int64_t rows, int64_t K, int8_t* q, float* s, uint64_t wait_limit_ns,
-                            cudaStream_t stream) {
-  const RqShape sh = rotquant_shape(static_cast<int>(K / 256));
-  const bool two_per_sm = 32 * (sh.warps + 1) <= 736;
-  switch (sh.gps) {
-    case 1:
-      return two_per_sm ? launch_rotquant_t<T, 1, 2>(x, rows, K, q, s, sh, wait_limit_ns, stream)
-                        : launch_rotquant_t<T, 1, 1>(x, rows, K, q, s, sh, wait_limit_ns, stream);
-    case 2: return launch_rotquant_t<T, 2, 1>(x, rows, K, q, s, sh, wait_limit_ns, stream);
-    case 3: return launch_rotquant_t<T, 3, 1>(x, rows, K, q, s, sh, wait_limit_ns, stream);
-    default: return launch_rotquant_t<T, 4, 1>(x, rows, K, q, s, sh, wait_limit_ns, stream);
+  if (sh.gps == 1) {
+    if (sh.small) rotquant_kernel<T, 1, true><<<grid, threads, smem, stream>>>(x, a);
+    else rotquant_kernel<T, 1, false><<<grid, threads, smem, stream>>>(x, a);
+  } else {
+    if (sh.small) rotquant_kernel<T, 2, true><<<grid, threads, smem, stream>>>(x, a);
+    else rotquant_kernel<T, 2, false><<<grid, threads, smem, stream>>>(x, a);
   }
+  return cudaGetLastError();
 }
 
 }  // namespace h3q
