@@ -1,18 +1,22 @@
 """Benchmark of the INT8 ConvRot hot path on B200.
 
-One step = one pass of the whole path over one batch of synthetic tokens: the
-FFN block (rotate + per-token quantize x, int8 GEMM against the [gate; up]
-weight with the fused SwiGLU epilogue, re-rotate + requantize h, int8 GEMM
-against the down weight with the fused rescale epilogue), i.e. every step of
-the method. Default workload: M = 16384 tokens, hidden K = 5376, FFN width
-F = 14336, activations N(0,1) with 1% outlier channels x50, weights N(0, 0.02)
+One step = one pass of the whole path over one batch of synthetic tokens. The
+default workload is the FFN block (every step of the method: rotate + per-token
+quantize x, int8 GEMM against the [gate; up] weight with the fused SwiGLU
+epilogue, re-rotate + requantize h, int8 GEMM against the down weight with the
+fused rescale epilogue) at M = 16384 tokens, hidden K = 5376, FFN width
+F = 14336; activations N(0,1) with 1% outlier channels x50, weights N(0, 0.02)
 prepared on the device by the library's own weight preparation.
 
-Headline value: int8 GEMM operations of the step (2*M*2F*K + 2*M*K*F) per
-second of device time, in TOPS. Also reported: FFN tokens/s, the
-rotate+quantize bandwidth, the dominant kernel's roofline fraction, an
-end-to-end number through host buffers, and the CPU oracle's rate on a bounded
-sample of the same workload.
+Headline value: int8 GEMM operations of the step per second of device time, in
+TOPS. Also reported: FFN tokens/s, the rotate+quantize bandwidth, the dominant
+kernel's roofline fraction, an end-to-end number through host buffers, and the
+CPU oracle's rate on a bounded sample of the same workload.
+
+Other workloads (--workload): qkv (4096 x 5376 -> 16128 with bias), out
+(32768 x 5376 -> 5376 with bias), tiny (64 x 512 -> 256), sweep (one denoising
+step's linear sweep: 50 blocks x (QKV, out, FFN) at 32768 tokens, about 17 GB of
+int8 weights resident, per-block activations generated before timing).
 
 Multi-GPU (torchrun): every rank runs its own batch with replicated weights
 (the rows are independent; there is no data-path collective). Times are the
@@ -35,17 +39,18 @@ sys.path.insert(0, ROOT)
 L2_FLUSH_BYTES = 256 << 20
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 GEMM_SRC = os.path.join(ROOT, "w8a8_rotation_quantized_b200", "csrc", "gemm_sm100.cuh")
+METRIC = "INT8 ConvRot linear TOPS"
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="h3q", choices=["h3q", "reference"])
-    ap.add_argument("--M", type=int, default=16384)
-    ap.add_argument("--K", type=int, default=5376)
-    ap.add_argument("--F", type=int, default=14336)
+    ap.add_argument("--workload", default="ffn", choices=["ffn", "qkv", "out", "tiny", "sweep"])
+    ap.add_argument("--M", type=int, default=None, help="tokens per GPU (default: the workload's)")
+    ap.add_argument("--F", type=int, default=None, help="FFN width (default 14336)")
     ap.add_argument("--kernel-reps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -53,25 +58,58 @@ def parse():
     return ap.parse_args()
 
 
-def gemm_ops(M, K, F):
-    return 2.0 * M * (2 * F) * K + 2.0 * M * K * F
+# ----------------------------------------------------------------------------- workloads
+class Spec:
+    """Shapes of one workload; ops() is the int8 GEMM work of one step."""
 
+    def __init__(self, name, M, K, N=None, F=None, bias=False, blocks=1):
+        self.name, self.M, self.K, self.N, self.F, self.bias, self.blocks = name, M, K, N, F, bias, blocks
 
-def workload_config(args, world):
-    return {
-        "workload": f"FFN block M={args.M} K={args.K} F={args.F}: rotquant(x) -> int8 GEMM [gate;up] + SwiGLU "
+    def ops(self, M=None):
+        M = self.M if M is None else M
+        if self.name == "ffn":
+            return 2.0 * M * (2 * self.F) * self.K + 2.0 * M * self.K * self.F
+        if self.name == "sweep":
+            per_block = 2.0 * M * self.K * (16128 + 5376) + 2.0 * M * (2 * self.F) * self.K + 2.0 * M * self.K * self.F
+            return per_block * self.blocks
+        return 2.0 * M * self.N * self.K
+
+    def describe(self, world):
+        d = {"ffn": f"FFN block M={self.M} K={self.K} F={self.F}: rotquant(x) -> int8 GEMM [gate;up] + SwiGLU "
                     f"-> rotquant(h) -> int8 GEMM down",
-        "tokens_per_gpu": args.M, "hidden": args.K, "ffn_width": args.F,
-        "global_batch_tokens": args.M * world, "parallelism": f"replicas x{world} (rows independent)",
-        "activations": "bf16 N(0,1), 1% outlier channels x50, seed 0",
-        "weights": "fp32 N(0,0.02) -> rotated per-row int8 on device, seed 0",
-        "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); inputs also exceed L2",
+             "qkv": f"QKV projection M={self.M} K={self.K} N={self.N} with bias: rotquant(x) -> int8 GEMM + rescale",
+             "out": f"attention-output projection M={self.M} K={self.K} N={self.N} with bias: rotquant(x) -> "
+                    f"int8 GEMM + rescale",
+             "tiny": f"tiny linear M={self.M} K={self.K} N={self.N}: rotquant(x) -> int8 GEMM + rescale",
+             "sweep": f"one denoising step's linear sweep: {self.blocks} blocks x (QKV {self.K}->16128, out "
+                      f"{self.K}->{self.K}, FFN {self.K}->2x{self.F}->{self.K}) at M={self.M}"}[self.name]
+        return {
+            "workload": d, "tokens_per_gpu": self.M, "hidden": self.K,
+            "global_batch_tokens": self.M * world, "parallelism": f"replicas x{world} (rows independent)",
+            "activations": "bf16 N(0,1), 1% outlier channels x50 (tiny: 4 channels x40), seed 0",
+            "weights": "fp32 N(0,0.02) -> rotated per-row int8 on device, seed 0",
+            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write); inputs also exceed L2",
+        }
+
+
+def make_spec(args):
+    F = args.F or 14336
+    table = {
+        "ffn": Spec("ffn", 16384, 5376, F=F),
+        "qkv": Spec("qkv", 4096, 5376, N=16128, bias=True),
+        "out": Spec("out", 32768, 5376, N=5376, bias=True),
+        "tiny": Spec("tiny", 64, 512, N=256),
+        "sweep": Spec("sweep", 32768, 5376, F=F, bias=True, blocks=50),
     }
+    s = table[args.workload]
+    if args.M is not None:
+        s.M = args.M
+    return s
 
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -82,12 +120,13 @@ class ClockSampler:
         try:
             self.path = f"/tmp/h3q_clocks_{os.getpid()}.csv"
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
+        """Summary of the samples taken between host times t0 and t1 (seconds)."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -95,53 +134,102 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
+        from datetime import datetime
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            if t0 is not None and not (t0 <= ts <= t1):
+                continue
+            rows.append(parts[1:])
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
         load = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
         return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(rows)}
 
 
 # ----------------------------------------------------------------------------- oracle rate
-def oracle_rate(M, K, F, target_s, threads_note=True):
-    """Times the CPU oracle's FFN on a bounded sample of rows of the same workload."""
+def _oracle_ffn_setup(K, F):
     import numpy as np
 
     import oracle
     import synth
 
-    wl_ids = synth.tensor_ids()
-    factors = synth.column_factors(K, synth.outlier_columns(0, wl_ids["outlier"], K, int(round(0.01 * K))), 50.0)
-    wgu = synth.weight_host(0, wl_ids["w_gu"], np.arange(2 * F), K)
-    wd = synth.weight_host(0, wl_ids["w_down"], np.arange(K), F)
-    qgu, sgu = oracle.prepare_weight(wgu)
-    qd, sd = oracle.prepare_weight(wd)
-    del wgu, wd
+    ids = synth.tensor_ids()
+    factors = synth.column_factors(K, synth.outlier_columns(0, ids["outlier"], K, int(round(0.01 * K))), 50.0)
+    qgu, sgu = oracle.prepare_weight(synth.weight_host(0, ids["w_gu"], np.arange(2 * F), K))
+    qd, sd = oracle.prepare_weight(synth.weight_host(0, ids["w_down"], np.arange(K), F))
+    return ids, factors, qgu, sgu, qd, sd
+
+
+def oracle_rate(spec, target_s):
+    """Times the CPU oracle's FFN (or linear layer) on a bounded sample of rows of the workload."""
+    import numpy as np
+
+    import oracle
+    import synth
+
+    K = spec.K
+    if spec.name in ("ffn", "sweep"):
+        ids, factors, qgu, sgu, qd, sd = _oracle_ffn_setup(K, spec.F)
+
+        def run(rows):
+            x = synth.activation_host(0, ids["x"], np.arange(rows), K, factors)
+            t0 = time.perf_counter()
+            oracle.ffn(x, qgu, sgu, qd, sd)
+            return time.perf_counter() - t0
+
+        def ops(rows):
+            return 2.0 * rows * (2 * spec.F) * K + 2.0 * rows * K * spec.F
+        what = "FFN"
+    else:
+        ids = synth.tensor_ids()
+        nout = 4 if spec.name == "tiny" else int(round(0.01 * K))
+        factors = synth.column_factors(K, synth.outlier_columns(0, ids["outlier"], K, nout),
+                                       40.0 if spec.name == "tiny" else 50.0)
+        wq, sw = oracle.prepare_weight(synth.weight_host(0, ids["w"], np.arange(spec.N), K))
+        b = synth.bias_host(0, ids["bias"], spec.N) if spec.bias else None
+
+        def run(rows):
+            x = synth.activation_host(0, ids["x"], np.arange(rows), K, factors)
+            t0 = time.perf_counter()
+            oracle.linear(x, wq, sw, bias_bits=b)
+            return time.perf_counter() - t0
+
+        def ops(rows):
+            return 2.0 * rows * spec.N * K
+        what = "linear layer"
     rows = 8
     while True:
-        x = synth.activation_host(0, wl_ids["x"], np.arange(rows), K, factors)
-        t0 = time.perf_counter()
-        oracle.ffn(x, qgu, sgu, qd, sd)
-        dt = time.perf_counter() - t0
-        if dt >= target_s or rows >= M:
+        dt = run(rows)
+        if dt >= target_s or rows >= spec.M:
             break
-        rows = min(M, max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 1.1)))
-    return {"value": gemm_ops(rows, K, F) / dt / 1e12, "unit": "TOPS", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"{rows} of {M} token rows of the same FFN workload (full weights), {dt:.1f} s"}
+        rows = min(spec.M, max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 1.1)))
+    return {"value": ops(rows) / dt / 1e12, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{rows} of {spec.M} token rows of the same {what} workload (full weights), {dt:.1f} s"}
 
 
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args):
+    """The oracle itself, timed on the host cores: there is no other reference
+    implementation (the reference is a set of pages, not code)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
@@ -151,34 +239,45 @@ def run_reference(args):
     import oracle
     import synth
 
-    K, F = args.K, args.F
-    ids = synth.tensor_ids()
-    factors = synth.column_factors(K, synth.outlier_columns(0, ids["outlier"], K, int(round(0.01 * K))), 50.0)
-    qgu, sgu = oracle.prepare_weight(synth.weight_host(0, ids["w_gu"], np.arange(2 * F), K))
-    qd, sd = oracle.prepare_weight(synth.weight_host(0, ids["w_down"], np.arange(K), F))
+    spec = make_spec(args)
+    if spec.name == "sweep":
+        spec = Spec("ffn", spec.M, spec.K, F=spec.F)  # the sweep's dominant layer
+    K = spec.K
+    if spec.name == "ffn":
+        ids, factors, qgu, sgu, qd, sd = _oracle_ffn_setup(K, spec.F)
+
+        def run(x):
+            oracle.ffn(x, qgu, sgu, qd, sd)
+    else:
+        ids = synth.tensor_ids()
+        factors = synth.column_factors(K, synth.outlier_columns(0, ids["outlier"], K, int(round(0.01 * K))), 50.0)
+        wq, sw = oracle.prepare_weight(synth.weight_host(0, ids["w"], np.arange(spec.N), K))
+        b = synth.bias_host(0, ids["bias"], spec.N) if spec.bias else None
+
+        def run(x):
+            oracle.linear(x, wq, sw, bias_bits=b)
     # rows per step: sized so that warmup + steps finish in about a minute of CPU time
     x = synth.activation_host(0, ids["x"], np.arange(8), K, factors)
     t0 = time.perf_counter()
-    oracle.ffn(x, qgu, sgu, qd, sd)
+    run(x)
     per_row = (time.perf_counter() - t0) / 8
-    rows = max(1, min(args.M, int(60.0 / max(1, args.steps + args.warmup) / per_row)))
+    rows = max(1, min(spec.M, int(60.0 / max(1, args.steps + args.warmup) / per_row)))
     x = synth.activation_host(0, ids["x"], np.arange(rows), K, factors)
     for _ in range(args.warmup):
-        oracle.ffn(x, qgu, sgu, qd, sd)
+        run(x)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.ffn(x, qgu, sgu, qd, sd)
+        run(x)
         times.append(time.perf_counter() - t0)
     dt = sum(times)
-    value = gemm_ops(rows, K, F) * args.steps / dt / 1e12
-    cfg = workload_config(args, world)
-    line = {"impl": "reference", "metric": "INT8 ConvRot linear TOPS", "value": value, "unit": "TOPS",
+    value = spec.ops(rows) * args.steps / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
-            "config": cfg,
+            "config": make_spec(args).describe(world),
             "cpu_baseline": {"value": value, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
-                             "sample": f"{rows} of {args.M} token rows per step, full weights"},
+                             "sample": f"{rows} of {spec.M} token rows per step, full weights"},
             "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -186,6 +285,8 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- GPU arm
 def traffic_from_profile(kernel_tag):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
+    or None once the kernel's source has changed since the counters were taken."""
     try:
         prof = json.load(open(PROFILE_TRAFFIC))
         src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()
@@ -204,6 +305,63 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+class Layer:
+    """Device tensors of one linear layer (x, prepared weight, bias); the codes,
+    scales and output may be shared between layers (`bufs`)."""
+
+    def __init__(self, h3q, synth, torch, dev, sp, M, K, N, tid_x, tid_w, tid_b, factors_dev, x_row0, bias,
+                 bufs=None):
+        self.M, self.K, self.N = M, K, N
+        self.x = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        synth.fill_device(0, tid_x, x_row0, M, K, self.x.data_ptr(), sp,
+                          factors_ptr=None if factors_dev is None else factors_dev.data_ptr(), bf16=True)
+        w = torch.empty((N, K), dtype=torch.float32, device=dev)
+        synth.fill_device(0, tid_w, 0, N, K, w.data_ptr(), sp, scale=float(synth.SIGMA_W), bf16=False)
+        self.wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        self.sw = torch.empty(N, dtype=torch.float32, device=dev)
+        h3q.h3q_prepare_weight(w, self.wq, self.sw)
+        del w
+        self.bias = None
+        if bias:
+            self.bias = torch.from_numpy(synth.bias_host(0, tid_b, N).view("int16")).to(dev).view(torch.bfloat16)
+        if bufs is None:
+            bufs = {"xq": torch.empty(M * K, dtype=torch.int8, device=dev),
+                    "sx": torch.empty(M, dtype=torch.float32, device=dev),
+                    "y": torch.empty(M * N, dtype=torch.bfloat16, device=dev)}
+        self.xq = bufs["xq"][:M * K].view(M, K)
+        self.sx = bufs["sx"][:M]
+        self.y = bufs["y"][:M * N].view(M, N)
+
+    def run(self, h3q, x=None):
+        h3q.h3q_rotate_quant(self.x if x is None else x, self.xq, self.sx)
+        h3q.h3q_linear_w8a8(self.xq, self.sx, self.wq, self.sw, self.y, bias=self.bias)
+
+
+class FFN:
+    """Device tensors of one FFN block."""
+
+    def __init__(self, h3q, synth, torch, dev, sp, M, K, F, tid_x, tid_gu, tid_d, factors_dev, x_row0, y=None):
+        self.M, self.K, self.F = M, K, F
+        self.x = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        synth.fill_device(0, tid_x, x_row0, M, K, self.x.data_ptr(), sp,
+                          factors_ptr=None if factors_dev is None else factors_dev.data_ptr(), bf16=True)
+        self.qgu = torch.empty((2 * F, K), dtype=torch.int8, device=dev)
+        self.sgu = torch.empty(2 * F, dtype=torch.float32, device=dev)
+        self.qd = torch.empty((K, F), dtype=torch.int8, device=dev)
+        self.sd = torch.empty(K, dtype=torch.float32, device=dev)
+        w = torch.empty((2 * F, K), dtype=torch.float32, device=dev)
+        synth.fill_device(0, tid_gu, 0, 2 * F, K, w.data_ptr(), sp, scale=float(synth.SIGMA_W), bf16=False)
+        h3q.h3q_prepare_weight(w, self.qgu, self.sgu)
+        w = torch.empty((K, F), dtype=torch.float32, device=dev)
+        synth.fill_device(0, tid_d, 0, K, F, w.data_ptr(), sp, scale=float(synth.SIGMA_W), bf16=False)
+        h3q.h3q_prepare_weight(w, self.qd, self.sd)
+        del w
+        self.y = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if y is None else y
+
+    def run(self, h3q, ws, x=None):
+        h3q.h3q_ffn(self.x if x is None else x, self.qgu, self.sgu, self.qd, self.sd, self.y, ws)
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -220,35 +378,67 @@ def run_gpu(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    M, K, F = args.M, args.K, args.F
-    ids = synth.tensor_ids()
+    spec = make_spec(args)
+    M, K = spec.M, spec.K
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
-
-    # ---- inputs, generated on the device; the weights prepared by the library
-    factors = synth.column_factors(K, synth.outlier_columns(0, ids["outlier"], K, int(round(0.01 * K))), 50.0)
+    ids = synth.tensor_ids()
+    nout = 4 if spec.name == "tiny" else int(round(0.01 * K))
+    factors = synth.column_factors(K, synth.outlier_columns(0, ids["outlier"], K, nout),
+                                   40.0 if spec.name == "tiny" else 50.0)
     fdev = torch.from_numpy(factors).to(dev)
-    x = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    # each rank takes its own rows of one long token stream
-    synth.fill_device(0, ids["x"], rank * M, M, K, x.data_ptr(), sp, factors_ptr=fdev.data_ptr(), bf16=True)
-    qgu = torch.empty((2 * F, K), dtype=torch.int8, device=dev)
-    sgu = torch.empty(2 * F, dtype=torch.float32, device=dev)
-    qd = torch.empty((K, F), dtype=torch.int8, device=dev)
-    sd = torch.empty(K, dtype=torch.float32, device=dev)
-    w = torch.empty((2 * F, K), dtype=torch.float32, device=dev)
-    synth.fill_device(0, ids["w_gu"], 0, 2 * F, K, w.data_ptr(), sp, scale=float(synth.SIGMA_W), bf16=False)
-    h3q.h3q_prepare_weight(w, qgu, sgu)
-    w = torch.empty((K, F), dtype=torch.float32, device=dev)
-    synth.fill_device(0, ids["w_down"], 0, K, F, w.data_ptr(), sp, scale=float(synth.SIGMA_W), bf16=False)
-    h3q.h3q_prepare_weight(w, qd, sd)
-    del w
-    ws = torch.empty(h3q.h3q_ffn_workspace_size(M, K, F), dtype=torch.uint8, device=dev)
-    y = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    ws_bytes = 0
+
+    # ---- inputs generated on the device; weights prepared by the library. Each
+    # rank takes its own rows of one long token stream.
+    if spec.name == "ffn":
+        ffn = FFN(h3q, synth, torch, dev, sp, M, K, spec.F, ids["x"], ids["w_gu"], ids["w_down"], fdev, rank * M)
+        ws_bytes = h3q.h3q_ffn_workspace_size(M, K, spec.F)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+        def step():
+            ffn.run(h3q, ws)
+        launches_per_step = 4
+        in_tensor, out_tensor = ffn.x, ffn.y
+    elif spec.name == "sweep":
+        # per block: its weights and its three input activations; codes, scales
+        # and outputs are shared by all blocks
+        bufs = {"xq": torch.empty(M * K, dtype=torch.int8, device=dev),
+                "sx": torch.empty(M, dtype=torch.float32, device=dev),
+                "y": torch.empty(M * 16128, dtype=torch.bfloat16, device=dev)}
+        y_ffn = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        blocks = []
+        for b in range(spec.blocks):
+            t = synth.tensor_ids(b)
+            fb = torch.from_numpy(synth.column_factors(K, synth.outlier_columns(0, t["outlier"], K, nout), 50.0)).to(dev)
+            qkv = Layer(h3q, synth, torch, dev, sp, M, K, 16128, t["x_qkv"], t["w_qkv"], t["b_qkv"], fb, rank * M,
+                        True, bufs)
+            out = Layer(h3q, synth, torch, dev, sp, M, K, K, t["x_out"], t["w_out"], t["b_out"], fb, rank * M,
+                        True, bufs)
+            ffn_b = FFN(h3q, synth, torch, dev, sp, M, K, spec.F, t["x_ffn"], t["w_gu"], t["w_down"], fb, rank * M,
+                        y_ffn)
+            blocks.append((qkv, out, ffn_b))
+            torch.cuda.synchronize()
+        ws_bytes = h3q.h3q_ffn_workspace_size(M, K, spec.F)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+        def step():
+            for qkv, out, ffn_b in blocks:
+                qkv.run(h3q)
+                out.run(h3q)
+                ffn_b.run(h3q, ws)
+        launches_per_step = 8 * spec.blocks
+        in_tensor, out_tensor = blocks[0][0].x, blocks[0][0].y
+    else:
+        layer = Layer(h3q, synth, torch, dev, sp, M, K, spec.N, ids["x"], ids["w"], ids["bias"], fdev, rank * M,
+                      spec.bias)
+
+        def step():
+            layer.run(h3q)
+        launches_per_step = 2
+        in_tensor, out_tensor = layer.x, layer.y
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
-
-    def step():
-        h3q.h3q_ffn(x, qgu, sgu, qd, sd, y, ws)
 
     def barrier():
         if world > 1:
@@ -262,42 +452,31 @@ def run_gpu(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
+    steps = args.steps if spec.name != "sweep" else max(1, min(args.steps, 5))
     for _ in range(args.warmup):
         step()
     barrier()
 
     clocks = ClockSampler(local)
-    clocks.start()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     barrier()
-    for i in range(args.steps):
+    clocks.start()
+    time.sleep(0.5)  # the sampler is running before the timed region starts
+    t_host0 = time.time()
+    for i in range(steps):
         flush.fill_(i & 0xFF)
         starts[i].record(stream)
         step()
         ends[i].record(stream)
     barrier()
-    clk = clocks.stop()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(sum(step_ms))
+    clk = clocks.stop(t_host0, time.time())
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)))
     st = h3q.h3q_get_device_status()
     if st != h3q.H3Q_OK:
         raise RuntimeError(f"device status after the timed region: {h3q.h3q_status_string(st)}")
 
     # ---- per-kernel device times (same stream, events around each launch, L2 flushed)
-    L = h3q.h3q_ffn_workspace_size  # noqa: F841
-    off = 0
-    def carve(nbytes, dtype, shape):
-        nonlocal off
-        t = ws[off:off + nbytes].view(dtype).view(*shape)
-        off = (off + nbytes + 255) // 256 * 256
-        return t
-    xq = carve(M * K, torch.int8, (M, K))
-    sx = carve(M * 4, torch.float32, (M,))
-    hbuf = carve(M * F * 2, torch.bfloat16, (M, F))
-    hq = carve(M * F, torch.int8, (M, F))
-    sh = carve(M * 4, torch.float32, (M,))
-
     def time_kernel(fn):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.kernel_reps)]
@@ -310,23 +489,59 @@ def run_gpu(args):
         torch.cuda.synchronize()
         return sum(a.elapsed_time(b) for a, b in ev) / len(ev)
 
-    t_rq_x = time_kernel(lambda: h3q.h3q_rotate_quant(x, xq, sx))
-    t_gu = time_kernel(lambda: h3q.h3q_linear_w8a8(xq, sx, qgu, sgu, hbuf, epilogue=h3q.H3Q_EPI_SWIGLU))
-    t_rq_h = time_kernel(lambda: h3q.h3q_rotate_quant(hbuf, hq, sh))
-    t_down = time_kernel(lambda: h3q.h3q_linear_w8a8(hq, sh, qd, sd, y))
+    peaks, peak_src = measured_peaks()
+    # int8 dense tensor rate on B200 is twice the bf16 rate (4.5 vs 2.25 PFLOP/s nominal)
+    i8_peak = 2.0 * peaks["bf16_tflops"]
+    kernels = {}
+    if spec.name in ("ffn", "sweep"):
+        f = ffn if spec.name == "ffn" else blocks[0][2]
+        F = spec.F
+        off = [0]
 
-    # ---- end to end through host buffers: H2D of x, the C-ABI call, D2H of y
+        def carve(nbytes, dtype, shape):
+            t = ws[off[0]:off[0] + nbytes].view(dtype).view(*shape)
+            off[0] = (off[0] + nbytes + 255) // 256 * 256
+            return t
+        xq = carve(M * K, torch.int8, (M, K))
+        sx = carve(M * 4, torch.float32, (M,))
+        hbuf = carve(M * F * 2, torch.bfloat16, (M, F))
+        hq = carve(M * F, torch.int8, (M, F))
+        sh = carve(M * 4, torch.float32, (M,))
+        kernels["rotate_quant_x"] = time_kernel(lambda: h3q.h3q_rotate_quant(f.x, xq, sx))
+        kernels["gemm_gate_up_swiglu"] = time_kernel(
+            lambda: h3q.h3q_linear_w8a8(xq, sx, f.qgu, f.sgu, hbuf, epilogue=h3q.H3Q_EPI_SWIGLU))
+        kernels["rotate_quant_h"] = time_kernel(lambda: h3q.h3q_rotate_quant(hbuf, hq, sh))
+        kernels["gemm_down"] = time_kernel(lambda: h3q.h3q_linear_w8a8(hq, sh, f.qd, f.sd, f.y))
+        dom_ops = 2.0 * M * (2 * F) * K
+        dom_ms = kernels["gemm_gate_up_swiglu"]
+        dom_name, dom_tag = "gemm_i8_kernel<SwiGLU> (FFN gate/up)", "gemm_i8_swiglu_ffn"
+        rq = {"x": (M * K * 3 + M * 4) / (kernels["rotate_quant_x"] * 1e-3) / 1e9,
+              "h": (M * F * 3 + M * 4) / (kernels["rotate_quant_h"] * 1e-3) / 1e9}
+    else:
+        kernels["rotate_quant_x"] = time_kernel(lambda: h3q.h3q_rotate_quant(layer.x, layer.xq, layer.sx))
+        kernels["gemm"] = time_kernel(
+            lambda: h3q.h3q_linear_w8a8(layer.xq, layer.sx, layer.wq, layer.sw, layer.y, bias=layer.bias))
+        dom_ops = 2.0 * M * spec.N * K
+        dom_ms = kernels["gemm"]
+        dom_name, dom_tag = "gemm_i8_kernel<BF16> (linear)", f"gemm_i8_bf16_{spec.name}"
+        rq = {"x": (M * K * 3 + M * 4) / (kernels["rotate_quant_x"] * 1e-3) / 1e9}
+
+    # ---- end to end through host buffers: H2D of x, the C-ABI calls, D2H of y
     e2e = None
-    if not args.no_e2e:
-        x_host = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
-        x_host.copy_(x)
-        y_host = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
-        x_dev = torch.empty_like(x)
-        e_steps = max(3, min(args.steps, 10))
+    if not args.no_e2e and spec.name != "sweep":
+        x_host = torch.empty(in_tensor.shape, dtype=torch.bfloat16, pin_memory=True)
+        x_host.copy_(in_tensor)
+        y_host = torch.empty(out_tensor.shape, dtype=torch.bfloat16, pin_memory=True)
+        x_dev = torch.empty_like(in_tensor)
+        e_steps = max(3, min(steps, 10))
+
         def e2e_step():
             x_dev.copy_(x_host, non_blocking=True)
-            h3q.h3q_ffn(x_dev, qgu, sgu, qd, sd, y, ws)
-            y_host.copy_(y, non_blocking=True)
+            if spec.name == "ffn":
+                ffn.run(h3q, ws, x=x_dev)
+            else:
+                layer.run(h3q, x=x_dev)
+            y_host.copy_(out_tensor, non_blocking=True)
         e2e_step()
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -336,44 +551,38 @@ def run_gpu(args):
         b.record(stream)
         barrier()
         e_ms = max_over_ranks(a.elapsed_time(b) / e_steps)
-        e2e = {"value": gemm_ops(M, K, F) * world / (e_ms * 1e-3) / 1e12, "unit": "TOPS",
-               "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * K * 2, "ms_per_step": e_ms}
+        e2e = {"value": spec.ops() * world / (e_ms * 1e-3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": in_tensor.numel() * 2, "d2h_bytes_per_step": out_tensor.numel() * 2,
+               "ms_per_step": e_ms}
 
     if rank == 0:
-        ms = total_ms / args.steps
-        value = gemm_ops(M, K, F) * world / (ms * 1e-3) / 1e12
-        peaks, peak_src = measured_peaks()
-        # int8 dense tensor rate on B200 is twice the bf16 rate (4.5 vs 2.25 PFLOP/s nominal)
-        i8_peak = 2.0 * peaks["bf16_tflops"]
-        gu_ops = 2.0 * M * (2 * F) * K
-        achieved = gu_ops / (t_gu * 1e-3) / 1e12
-        traffic = traffic_from_profile("gemm_i8_swiglu_ffn")
-        rq_bytes = M * K * 3 + M * 4
+        ms = total_ms / steps
+        value = spec.ops() * world / (ms * 1e-3) / 1e12
+        achieved = dom_ops / (dom_ms * 1e-3) / 1e12
         line = {
-            "metric": "INT8 ConvRot linear TOPS", "value": value, "unit": "TOPS", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
-            "config": workload_config(args, world),
-            "ffn_tokens_per_s": M * world / (ms * 1e-3),
+            "config": spec.describe(world),
             "int8_peak_tops": i8_peak,
             "frac_of_int8_peak": value / i8_peak,
-            "kernels_ms": {"rotate_quant_x": t_rq_x, "gemm_gate_up_swiglu": t_gu, "rotate_quant_h": t_rq_h,
-                           "gemm_down": t_down},
-            "rotquant_gbs": {"x": rq_bytes / (t_rq_x * 1e-3) / 1e9,
-                             "h": (M * F * 3 + M * 4) / (t_rq_h * 1e-3) / 1e9,
-                             "peak": peaks["hbm_gbs"]},
-            "roofline": {"bound": "tensor", "kernel": "gemm_i8_kernel<SwiGLU> (gate/up)",
+            "kernels_ms": kernels,
+            "rotquant_gbs": dict(rq, peak=peaks["hbm_gbs"]),
+            "roofline": {"bound": "tensor", "kernel": dom_name,
                          "achieved": achieved, "peak": i8_peak, "unit": "TOPS",
-                         "frac": achieved / i8_peak, "traffic": traffic,
+                         "frac": achieved / i8_peak, "traffic": traffic_from_profile(dom_tag),
                          "peak_source": f"{peak_src}: 2 x bf16 burst {peaks['bf16_tflops']} TFLOP/s "
                                         "(int8 dense rate = 2 x bf16 on B200)"},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": launches_per_step * steps,
             "clocks": clk,
             "e2e": e2e,
         }
+        if spec.name in ("ffn", "sweep"):
+            line["ffn_tokens_per_s"] = M * world / (ms * 1e-3) * (1 if spec.name == "ffn" else 1.0 / spec.blocks)
         if not args.no_cpu_baseline:
             try:
-                line["cpu_baseline"] = oracle_rate(M, K, F, args.cpu_seconds)
+                line["cpu_baseline"] = oracle_rate(spec if spec.name != "sweep" else Spec("ffn", M, K, F=spec.F),
+                                                   args.cpu_seconds)
             except Exception as exc:  # the line still prints; the reason is kept
                 line["cpu_baseline"] = {"value": None, "error": repr(exc)}
         print(json.dumps(line), flush=True)

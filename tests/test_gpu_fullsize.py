@@ -118,3 +118,54 @@ def test_ffn_fullsize(h3q, cuda_device):
     assert np.array_equal(sh[msd].cpu().numpy().view(np.uint32), osh.view(np.uint32))
     got = bits(y[msd])
     assert np.array_equal(got, oy), f"{(got != oy).sum()} of {got.size} outputs differ"
+
+
+@pytest.mark.parametrize("block", [0, 49])
+def test_sweep_block_fullsize(h3q, cuda_device, block):
+    """One block of a denoising step's linear sweep at 32768 tokens: QKV and out
+    projections with bias and the FFN, each with its own per-block tensors."""
+    from _gpu_util import bits, dev_activation, dev_bias, dev_weight, sample_indices
+    dev = cuda_device
+    M, K, F = 32768, 5376, 14336
+    t = synth.tensor_ids(block)
+    f = synth.column_factors(K, synth.outlier_columns(0, t["outlier"], K, int(round(0.01 * K))), 50.0)
+    rng = np.random.default_rng(100 + block)
+    ms = sample_indices(M, 4, rng, must=(M - 1,))
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    sx = torch.empty(M, dtype=torch.float32, device=dev)
+    for name, N in (("qkv", 16128), ("out", K)):
+        x = dev_activation(0, t["x_" + name], M, K, f, dev)
+        w = dev_weight(0, t["w_" + name], N, K, dev)
+        wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        sw = torch.empty(N, dtype=torch.float32, device=dev)
+        h3q.h3q_prepare_weight(w, wq, sw)
+        del w
+        bias = dev_bias(0, t["b_" + name], N, dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        h3q.h3q_rotate_quant(x, xq, sx)
+        h3q.h3q_linear_w8a8(xq, sx, wq, sw, y, bias=bias)
+        torch.cuda.synchronize()
+        ns = sample_indices(N, 32, rng)
+        owq, osw = oracle.prepare_weight(synth.weight_host(0, t["w_" + name], ns, K))
+        oy, _ = oracle.linear(synth.activation_host(0, t["x_" + name], ms, K, f), owq, osw,
+                              bias_bits=synth.bias_host(0, t["b_" + name], N)[ns])
+        got = bits(y[torch.from_numpy(ms).to(dev)][:, torch.from_numpy(ns).to(dev)])
+        assert np.array_equal(got, oy), f"block {block} {name}: {(got != oy).sum()} of {got.size} differ"
+        del x, wq, y
+    x = dev_activation(0, t["x_ffn"], M, K, f, dev)
+    qgu = torch.empty((2 * F, K), dtype=torch.int8, device=dev)
+    sgu = torch.empty(2 * F, dtype=torch.float32, device=dev)
+    qd = torch.empty((K, F), dtype=torch.int8, device=dev)
+    sd = torch.empty(K, dtype=torch.float32, device=dev)
+    h3q.h3q_prepare_weight(dev_weight(0, t["w_gu"], 2 * F, K, dev), qgu, sgu)
+    h3q.h3q_prepare_weight(dev_weight(0, t["w_down"], K, F, dev), qd, sd)
+    ws = torch.empty(h3q.h3q_ffn_workspace_size(M, K, F), dtype=torch.uint8, device=dev)
+    y = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    h3q.h3q_ffn(x, qgu, sgu, qd, sd, y, ws)
+    torch.cuda.synchronize()
+    assert h3q.h3q_get_device_status() == h3q.H3Q_OK
+    ogu, osgu = oracle.prepare_weight(synth.weight_host(0, t["w_gu"], np.arange(2 * F), K))
+    od, osd = oracle.prepare_weight(synth.weight_host(0, t["w_down"], np.arange(K), F))
+    oy, _, _, _ = oracle.ffn(synth.activation_host(0, t["x_ffn"], ms, K, f), ogu, osgu, od, osd)
+    got = bits(y[torch.from_numpy(ms).to(dev)])
+    assert np.array_equal(got, oy), f"block {block} ffn: {(got != oy).sum()} of {got.size} differ"

@@ -24,8 +24,9 @@
 //               tcgen05.ld, fp32 rescale, bias, bf16 (or SwiGLU), stores; then
 //               they free the accumulator on the leader's barrier.
 // Two 256-column accumulators let the epilogue of tile i overlap the main loop
-// of tile i+1. Tiles are walked in groups of GROUP_M row blocks so the weight
-// blocks in flight stay in L2. No load uses cluster multicast.
+// of tile i+1. Tiles are walked in groups of row blocks (the group's A tiles are
+// reused from L2 by every N block; each B tile is read once per group). No load
+// uses cluster multicast.
 //
 // SwiGLU: the B tile of an output tile holding h columns [j0, j0+128) stacks
 // gate rows [j0, j0+128) (in the leader) over up rows [F+j0, F+j0+128) (in the
@@ -54,7 +55,6 @@ constexpr int kAStage = kBM * kBK;  // 16 KB
 constexpr int kBStage = 128 * kBK;  // 16 KB: this CTA's half of the B tile
 constexpr int kTmemCols = 512;
 constexpr int kGemmThreads = 320;  // producer, MMA, 8 epilogue warps
-constexpr int kGroupM = 8;  // pair tiles (256 rows each) per raster group
 constexpr size_t kGemmSmem =
     size_t(kStages) * (kAStage + kBStage) + 1024 /*align*/ + 256 /*barriers*/ + 4 * kBN * 4 /*column scales, biases*/;
 
@@ -65,6 +65,9 @@ struct GemmParams {
   int N;            // output columns (SwiGLU: F)
   int K;
   int num_m, num_n, num_tiles;
+  int raster;       // tile order: see tile_coords
+  int group_m;      // pair-row blocks per group (raster 0)
+  int pol_a, pol_b; // L2 policy of the A and B tile loads: 0 evict-first, 1 evict-last, 2 evict-normal
   int b_row_up;     // SwiGLU: first up row of B (= F)
   const float* sx;  // [M]
   const float* sw;  // [N] (SwiGLU: [2F])
@@ -73,11 +76,20 @@ struct GemmParams {
   uint64_t wait_limit_ns;
 };
 
-__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
-  const int per_group = kGroupM * num_n;
+// Tile order. raster 0: groups of group_m pair-row blocks; within a group the
+// row blocks vary fastest, so the group's A tiles are reused from L2 by every N
+// block and each B tile is read once per group. raster 1: all row blocks of one
+// N block before the next N block.
+__device__ __forceinline__ void tile_coords(int tile, const GemmParams& p, int& mb, int& nb) {
+  if (p.raster == 1) {
+    mb = tile % p.num_m;
+    nb = tile / p.num_m;
+    return;
+  }
+  const int per_group = p.group_m * p.num_n;
   const int gid = tile / per_group;
-  const int first_m = gid * kGroupM;
-  const int gm = min(num_m - first_m, kGroupM);
+  const int first_m = gid * p.group_m;
+  const int gm = min(p.num_m - first_m, p.group_m);
   const int r = tile - gid * per_group;
   mb = first_m + r % gm;
   nb = r / gm;
@@ -181,14 +193,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer (both CTAs)
-      const uint64_t pol = policy_evict_last();
+      auto policy = [](int k) {
+        return k == 0 ? policy_evict_first() : (k == 1 ? policy_evict_last() : policy_evict_normal());
+      };
+      const uint64_t pol_a = policy(p.pol_a);
+      const uint64_t pol_b = policy(p.pol_b);
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
         int mb, nb;
-        tile_coords(tile, p.num_m, p.num_n, mb, nb);
+        tile_coords(tile, p, mb, nb);
         const int a_row = mb * (2 * kBM) + static_cast<int>(rank) * kBM;
         const int b_row = (EPI == kEpiSwiGLU) ? (rank == 0 ? nb * 128 : p.b_row_up + nb * 128)
                                               : nb * kBN + static_cast<int>(rank) * 128;
@@ -199,8 +215,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
           const uint32_t full_leader = cluster_map(&full[stage], 0);
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (kAStage + kBStage));
-          tma_load_2d_pair(sA + stage * kAStage, &tmA, full_leader, kb * kBK, a_row, pol);
-          tma_load_2d_pair(sB + stage * kBStage, &tmB, full_leader, kb * kBK, b_row, pol);
+          tma_load_2d_pair(sA + stage * kAStage, &tmA, full_leader, kb * kBK, a_row, pol_a);
+          tma_load_2d_pair(sB + stage * kBStage, &tmB, full_leader, kb * kBK, b_row, pol_b);
           ++issued;
           if (++stage == kStages) {
             stage = 0;
@@ -276,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     int iter = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs, ++iter) {
       int mb, nb;
-      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(tile, p, mb, nb);
       float* cs = col_scale + (iter & 1) * kBN;  // this tile's 256 column scales ...
       float* cb = col_bias + (iter & 1) * kBN;   // ... and biases, staged once per tile
       if constexpr (EPI != kEpiS32) {

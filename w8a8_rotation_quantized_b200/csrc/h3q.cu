@@ -19,6 +19,20 @@ using h3q::GemmParams;
 
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 
+// GEMM tile order and L2 policies (0 evict-first, 1 evict-last, 2 evict-normal).
+#ifndef H3Q_GEMM_GROUP_ROWS
+#define H3Q_GEMM_GROUP_ROWS 16
+#endif
+#ifndef H3Q_GEMM_POLICY_A
+#define H3Q_GEMM_POLICY_A 1
+#endif
+#ifndef H3Q_GEMM_POLICY_B
+#define H3Q_GEMM_POLICY_B 1
+#endif
+constexpr int kGemmGroupRows = H3Q_GEMM_GROUP_ROWS;
+constexpr int kGemmPolicyA = H3Q_GEMM_POLICY_A;
+constexpr int kGemmPolicyB = H3Q_GEMM_POLICY_B;
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -72,7 +86,7 @@ h3q_status launch_gemm(const int8_t* a, const int8_t* b, int64_t M, int64_t K, i
                                     static_cast<int>(h3q::kGemmSmem));
   });
   if (attr_err != cudaSuccess) return H3Q_ERR_CUDA;
-  GemmParams p;
+  GemmParams p{};
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N_out);
   p.K = static_cast<int>(K);
@@ -81,6 +95,13 @@ h3q_status launch_gemm(const int8_t* a, const int8_t* b, int64_t M, int64_t K, i
                                      : static_cast<int>((N_out + h3q::kBN - 1) / h3q::kBN);
   p.num_tiles = p.num_m * p.num_n;
   p.b_row_up = (EPI == h3q::kEpiSwiGLU) ? static_cast<int>(N_out) : 0;
+  // Tile order: groups of kGemmGroupRows pair-row blocks (the group's A tiles are
+  // reused by every N block from L2, each B tile is read once per group); both
+  // operands are loaded with an evict-last L2 policy.
+  p.raster = 0;
+  p.group_m = kGemmGroupRows < p.num_m ? kGemmGroupRows : p.num_m;
+  p.pol_a = kGemmPolicyA;
+  p.pol_b = kGemmPolicyB;
   p.sx = sx;
   p.sw = sw;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
