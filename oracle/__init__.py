@@ -54,6 +54,7 @@ def _load():
             "orc_linear": (I64, [P, I64, I64, P, P, I64, P, ctypes.c_int, P, P, P, P, P]),
             "orc_ffn": (I64, [P, I64, I64, P, P, P, I64, P, P, P, P, P, P, P]),
             "orc_num_threads": (ctypes.c_int, []),
+            "orc_lora_merge": (None, [P, P, I64, I64, P, P, I64, F]),
             "orc_f32_to_bf16": (ctypes.c_uint16, [F]),
             "orc_bf16_to_f32": (F, [ctypes.c_uint16]),
         }
@@ -211,6 +212,20 @@ def linear(x_bits, wq, sw, bias_bits=None, swiglu_epilogue=False, want=()):
         if arr is not None:
             extra[name] = arr
     return y, extra
+
+
+def lora_merge(wq, sw, lora_a, lora_b, alpha):
+    """LoRA merge: (wq, sw) rotated int8 rows plus alpha * B A, A rotated along K,
+    requantized per row. Returns new (wq, sw); the inputs are not modified."""
+    q = np.array(wq, dtype=np.int8, copy=True, order="C")
+    s = np.array(sw, dtype=np.float32, copy=True, order="C")
+    a = _c(lora_a, np.float32)
+    b = _c(lora_b, np.float32)
+    N, K = q.shape
+    r = a.shape[0]
+    assert a.shape == (r, K) and b.shape == (N, r) and K % 256 == 0
+    _load().orc_lora_merge(_p(q), _p(s), N, K, _p(a), _p(b), r, float(alpha))
+    return q, s
 
 
 def ffn(x_bits, w_gu, s_gu, w_down, s_down, b_gu=None, b_down=None):

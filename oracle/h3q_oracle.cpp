@@ -18,6 +18,9 @@
 //  * The FFN-output projection stays INT8 ConvRot, so the SwiGLU output is
 //    rotated and quantized again before it (Minimax_h3_hybrid model card,
 //    "Checkpoints").
+//  * LoRA deltas are merged into the stored int8 weights at load by
+//    dequantizing, adding and requantizing (h3-rs README, "Speed", "What makes
+//    it fast"); the delta is rotated along K like the weights it joins.
 //
 // Readings where the pages are silent (each one is listed with its reason in
 // the design notes): H is the natural-order Sylvester matrix scaled by 1/16; the
@@ -26,7 +29,10 @@
 // one scale per token over the whole row; epilogue order
 // ((float)acc * sx) * sw + bias without fused multiply-add; SwiGLU takes the
 // first half of the fc1 outputs as gate and the second half as up; e^-g is
-// evaluated by Cody-Waite reduction and a degree-7 Taylor polynomial in fp32.
+// evaluated by Cody-Waite reduction and a degree-7 Taylor polynomial in fp32;
+// the LoRA delta B A_rot is a fused multiply-add chain over the rank index in
+// ascending order, scaled by alpha and added to q * s as two rounded products
+// and one rounded add.
 //
 // Plain loops, no blocking or fusion beyond what the definition states.
 // Build: g++ -O2 -std=c++17 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC
@@ -291,6 +297,35 @@ int64_t orc_ffn(const uint16_t* x, int64_t M, int64_t K, const int8_t* w_gu, con
   if (hq_out) std::memcpy(hq_out, hq.data(), hq.size());
   if (sh_out) std::memcpy(sh_out, sh.data(), sh.size() * 4);
   return overflow;
+}
+
+// ---------------------------------------------------------------------------
+// LoRA merge into stored rotated int8 weights (h3-rs README, "What makes it
+// fast": LoRAs are merged into the int8 weights at load: dequantize, add,
+// requantize). The stored codes are in the rotated basis, so the low-rank delta
+// alpha * B A (B [N, r], A [r, K] in the model's basis) is rotated along K the
+// same way: A_rot = A blockdiag(H/16), delta = alpha * B A_rot. Per element, in
+// fp32 and in this order: d = sum over j ascending of B[n][j] * A_rot[j][k] as a
+// fused multiply-add chain from 0; w = (float)q * s + alpha * d (two rounded
+// products, one rounded add); then each row is requantized like a weight row
+// (step 5 without the rotation). Updates q and s in place.
+// ---------------------------------------------------------------------------
+void orc_lora_merge(int8_t* q, float* s, int64_t N, int64_t K, const float* lora_a, const float* lora_b,
+                    int64_t r, float alpha) {
+  std::vector<float> a_rot(size_t(r) * K);
+  orc_rotate_f32(lora_a, r, K, a_rot.data());
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    std::vector<float> w(K);
+    for (int64_t k = 0; k < K; ++k) {
+      float d = 0.0f;
+      for (int64_t j = 0; j < r; ++j) d = std::fma(lora_b[n * r + j], a_rot[j * K + k], d);
+      const float base = float(q[n * K + k]) * s[n];
+      const float delta = alpha * d;
+      w[k] = base + delta;
+    }
+    quantize_row(w.data(), K, q + n * K, s + n);
+  }
 }
 
 int orc_num_threads(void) {

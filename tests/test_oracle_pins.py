@@ -325,3 +325,51 @@ def test_ffn_accuracy_vs_unquantized():
     # h's codes are its own rotation + quantization
     q2, s2 = oracle.rotate_quant_bf16(h)
     assert np.array_equal(q2, hq) and np.array_equal(s2, sh)
+
+
+# ------------------------------------------------------------------- LoRA merge
+def _lora(N, K, r, seed=3):
+    rng = np.random.default_rng(seed)
+    a = (rng.standard_normal((r, K)) * 0.05).astype(np.float32)
+    b = (rng.standard_normal((N, r)) * 0.05).astype(np.float32)
+    return a, b
+
+
+def test_lora_merge_zero_delta_keeps_codes():
+    w = synth.weight_fp32(0, 2, np.arange(64), 512)
+    wq, sw = oracle.prepare_weight(w)
+    a, b = _lora(64, 512, 8)
+    q2, s2 = oracle.lora_merge(wq, sw, a, b, 0.0)
+    assert np.array_equal(q2, wq)
+    assert np.array_equal(s2, sw)
+    q3, s3 = oracle.lora_merge(wq, sw, a, np.zeros_like(b), 1.5)
+    assert np.array_equal(q3, wq) and np.array_equal(s3, sw)
+
+
+def test_lora_merge_matches_rotated_sum_within_quantization_error():
+    N, K, r, alpha = 96, 768, 16, 0.75
+    w = synth.weight_fp32(0, 2, np.arange(N), K)
+    wq, sw = oracle.prepare_weight(w)
+    a, b = _lora(N, K, r)
+    q2, s2 = oracle.lora_merge(wq, sw, a, b, alpha)
+    H = kron_hadamard().astype(np.float64) / 16.0
+    rot = lambda m: np.einsum("rgj,ij->rgi", m.reshape(m.shape[0], -1, 256), H).reshape(m.shape)
+    target = wq.astype(np.float64) * sw[:, None] + alpha * (b.astype(np.float64) @ rot(a.astype(np.float64)))
+    err = np.abs(q2.astype(np.float64) * s2[:, None] - target)
+    assert np.all(err <= s2[:, None] * (0.5 + 1e-4))
+    assert np.all(np.abs(q2).max(axis=1) == 127)
+    # the delta is applied in the rotated basis: the unrotated sum is far off
+    wrong = wq.astype(np.float64) * sw[:, None] + alpha * (b.astype(np.float64) @ a.astype(np.float64))
+    assert np.abs(q2.astype(np.float64) * s2[:, None] - wrong).max() > 10 * s2.max()
+
+
+def test_lora_merged_layer_matches_fp64_model():
+    N, K, r, alpha = 128, 512, 8, 1.0
+    x = synth.activation_bf16(0, 1, np.arange(48), K)
+    w = synth.weight_fp32(0, 2, np.arange(N), K)
+    wq, sw = oracle.prepare_weight(w)
+    a, b = _lora(N, K, r)
+    q2, s2 = oracle.lora_merge(wq, sw, a, b, alpha)
+    y, _ = oracle.linear(x, q2, s2)
+    ref = f32(x).astype(np.float64) @ (w.astype(np.float64) + alpha * b.astype(np.float64) @ a.astype(np.float64)).T
+    assert np.linalg.norm(f32(y) - ref) / np.linalg.norm(ref) <= 2e-2
