@@ -18,6 +18,10 @@ Other workloads (--workload): qkv (4096 x 5376 -> 16128 with bias), out
 step's linear sweep: 50 blocks x (QKV, out, FFN) at 32768 tokens, about 17 GB of
 int8 weights resident, per-block activations generated before timing).
 
+Workload lora: merging a rank-64 LoRA at load into one FFN block's int8
+weights (gate/up [28672, 5376] and down [5376, 14336]); value in fp32 TFLOP/s of
+the merge's low-rank product, bound by the fp32 FMA pipe.
+
 Multi-GPU (torchrun): every rank runs its own batch with replicated weights
 (the rows are independent; there is no data-path collective). Times are the
 max over ranks; the value is the work of all ranks over that time.
@@ -48,7 +52,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="h3q", choices=["h3q", "reference"])
-    ap.add_argument("--workload", default="ffn", choices=["ffn", "qkv", "out", "tiny", "sweep"])
+    ap.add_argument("--workload", default="ffn", choices=["ffn", "qkv", "out", "tiny", "sweep", "lora"])
     ap.add_argument("--M", type=int, default=None, help="tokens per GPU (default: the workload's)")
     ap.add_argument("--F", type=int, default=None, help="FFN width (default 14336)")
     ap.add_argument("--kernel-reps", type=int, default=10)
@@ -239,6 +243,23 @@ def run_reference(args):
     import oracle
     import synth
 
+    if args.workload == "lora":
+        per_step = 60.0 / max(1, args.steps + args.warmup)
+        for _ in range(args.warmup):
+            oracle_lora_rate(per_step)
+        vals = [oracle_lora_rate(per_step) for _ in range(args.steps)]
+        value = sum(v["rows"] for v in vals) * 2.0 * 5376 * synth.WORKLOADS["lora"].rank / \
+            sum(v["seconds"] for v in vals) / 1e12
+        line = {"impl": "reference", "metric": "LoRA merge TFLOP/s", "value": value, "unit": "TFLOP/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * sum(v["seconds"] for v in vals) / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": "LoRA merge at load into the gate/up weight, sampled rows"},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                                 "sample": vals[-1]["sample"]},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
     spec = make_spec(args)
     if spec.name == "sweep":
         spec = Spec("ffn", spec.M, spec.K, F=spec.F)  # the sweep's dominant layer
@@ -309,13 +330,15 @@ def job_tops(ops_per_rank_step, world, ms_per_step):
 
 # ----------------------------------------------------------------------------- GPU arm
 def traffic_from_profile(kernel_tag):
-    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
-    or None once the kernel's source has changed since the counters were taken."""
+    """DRAM bytes per launch of a kernel from a committed ncu summary, or None
+    once the kernel's source file has changed since the counters were taken."""
     try:
         prof = json.load(open(PROFILE_TRAFFIC))
-        src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()
         ent = prof.get(kernel_tag)
-        if ent and ent.get("source_sha256") == src_hash:
+        if not ent:
+            return None
+        src = os.path.join(ROOT, ent.get("source_file", os.path.relpath(GEMM_SRC, ROOT)))
+        if ent.get("source_sha256") == hashlib.sha256(open(src, "rb").read()).hexdigest():
             return ent.get("bytes_per_launch")
     except Exception:
         pass
@@ -384,6 +407,202 @@ class FFN:
 
     def run(self, h3q, ws, x=None):
         h3q.h3q_ffn(self.x if x is None else x, self.qgu, self.sgu, self.qd, self.sd, self.y, ws)
+
+
+def fp32_fma_peak_tflops(sms, sm_mhz):
+    """fp32 peak of the CUDA cores: 128 FMA lanes per SM, 2 flops per FMA."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def _lora_shapes(wl):
+    """(name, N, K) of the weights one LoRA step merges into."""
+    return [("gate_up", 2 * wl.F, wl.K), ("down", wl.K, wl.F)]
+
+
+def run_lora(args):
+    """LoRA merge at load: one step merges a rank-r LoRA into both int8 weights of
+    an FFN block, in place (rotate A, then the merge kernel, per weight)."""
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import w8a8_rotation_quantized_b200 as h3q
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    wl = synth.WORKLOADS["lora"]
+    r, alpha = wl.rank, wl.alpha
+    ids = synth.tensor_ids()
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    mats = []
+    for (name, N, K), (ta, tb, tw) in zip(_lora_shapes(wl), [("lora_a", "lora_b", "w_gu"),
+                                                           ("lora_a_down", "lora_b_down", "w_down")]):
+        w = torch.empty((N, K), dtype=torch.float32, device=dev)
+        synth.fill_device(wl.seed, ids[tw], 0, N, K, w.data_ptr(), sp, scale=float(synth.SIGMA_W), bf16=False)
+        wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        sw = torch.empty(N, dtype=torch.float32, device=dev)
+        h3q.h3q_prepare_weight(w, wq, sw)
+        del w
+        a = torch.empty((r, K), dtype=torch.float32, device=dev)
+        b = torch.empty((N, r), dtype=torch.float32, device=dev)
+        synth.fill_device(wl.seed, ids[ta], 0, r, K, a.data_ptr(), sp, scale=float(synth.SIGMA_W), bf16=False)
+        synth.fill_device(wl.seed, ids[tb], 0, N, r, b.data_ptr(), sp, scale=float(synth.SIGMA_W), bf16=False)
+        ws = torch.empty(h3q.h3q_lora_workspace_size(r, K), dtype=torch.uint8, device=dev)
+        mats.append(dict(name=name, N=N, K=K, wq=wq, sw=sw, a=a, b=b, ws=ws))
+    flops = sum(2.0 * m["N"] * m["K"] * r for m in mats)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    def merge(m, a=None, b=None):
+        h3q.h3q_lora_merge(m["wq"], m["sw"], m["a"] if a is None else a, m["b"] if b is None else b, alpha, m["ws"])
+
+    def step():
+        for m in mats:
+            merge(m)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    steps = max(1, min(args.steps, 50))
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    clocks = ClockSampler(local)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier()
+    clocks.start()
+    time.sleep(0.5)
+    t_host0 = time.time()
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    barrier()
+    clk = clocks.stop(t_host0, time.time())
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), dev)
+    st = h3q.h3q_get_device_status()
+    if st != h3q.H3Q_OK:
+        raise RuntimeError(f"device status after the timed region: {h3q.h3q_status_string(st)}")
+
+    kernels = {}
+    for m in mats:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.kernel_reps)]
+        for e0, e1 in ev:
+            flush.fill_(1)
+            e0.record(stream)
+            merge(m)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        kernels["merge_" + m["name"]] = sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
+
+    # end to end: the factors come from pinned host memory each step and the new
+    # scales go back; the weights stay resident (they are the model's).
+    e2e = None
+    if not args.no_e2e:
+        host = [(torch.empty(m["a"].shape, dtype=torch.float32, pin_memory=True).copy_(m["a"]),
+                 torch.empty(m["b"].shape, dtype=torch.float32, pin_memory=True).copy_(m["b"]),
+                 torch.empty(m["sw"].shape, dtype=torch.float32, pin_memory=True)) for m in mats]
+        dev_ab = [(torch.empty_like(m["a"]), torch.empty_like(m["b"])) for m in mats]
+        e_steps = max(4, min(steps, 12))
+        barrier()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(e_steps):
+            for m, (ha, hb, hs), (da, db) in zip(mats, host, dev_ab):
+                da.copy_(ha, non_blocking=True)
+                db.copy_(hb, non_blocking=True)
+                merge(m, da, db)
+                hs.copy_(m["sw"], non_blocking=True)
+        t1.record(stream)
+        barrier()
+        e_ms = max_over_ranks(t0.elapsed_time(t1) / e_steps, dev)
+        e2e = {"value": flops * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(m["a"].numel() * 4 + m["b"].numel() * 4 for m in mats),
+               "d2h_bytes_per_step": sum(m["sw"].numel() * 4 for m in mats), "ms_per_step": e_ms,
+               "steps": e_steps, "how": "factors copied from pinned host memory, scales read back, one stream"}
+
+    if rank == 0:
+        ms = total_ms / steps
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        sm_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
+        peak = fp32_fma_peak_tflops(sms, sm_mhz)
+        dom = max(mats, key=lambda m: m["N"] * m["K"])
+        dom_ms = kernels["merge_" + dom["name"]]
+        achieved = 2.0 * dom["N"] * dom["K"] * r / (dom_ms * 1e-3) / 1e12
+        line = {
+            "metric": "LoRA merge TFLOP/s", "value": flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"LoRA merge at load, rank {r}, alpha {alpha}, into one FFN block's int8 "
+                                   f"weights: " + ", ".join(f"{m['name']} [{m['N']}, {m['K']}]" for m in mats),
+                       "factors": "A [r, K] and B [N, r] fp32 N(0, 0.02), seed 0; weights fp32 N(0, 0.02) "
+                                  "prepared on device",
+                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+                       "parallelism": f"replicas x{world}"},
+            "kernels_ms": kernels,
+            "hbm_bytes_per_step": sum(2 * m["N"] * m["K"] + 8 * m["N"] + 8 * r * m["K"] + 4 * m["N"] * r
+                                      for m in mats),
+            "roofline": {"bound": "alu", "kernel": f"lora_merge_kernel ({dom['name']})", "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "traffic": traffic_from_profile("lora_merge_" + dom["name"]),
+                         "peak_source": f"derived: {sms} SMs x 128 fp32 FMA lanes x 2 flops x {sm_mhz} MHz "
+                                        "(max SM clock)"},
+            "gpu_launches": 2 * len(mats) * steps,
+            "clocks": clk,
+            "e2e": e2e,
+        }
+        if not args.no_cpu_baseline:
+            try:
+                line["cpu_baseline"] = oracle_lora_rate(args.cpu_seconds)
+            except Exception as exc:
+                line["cpu_baseline"] = {"value": None, "error": repr(exc)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def oracle_lora_rate(target_s, steps=None):
+    """The oracle's LoRA merge on a bounded sample of the gate/up weight's rows
+    (full K and rank); flops of the low-rank product per second."""
+    import numpy as np
+
+    import oracle
+    import synth
+    wl = synth.WORKLOADS["lora"]
+    ids = synth.tensor_ids()
+    N, K = _lora_shapes(wl)[0][1:]
+    r = wl.rank
+    a = synth.weight_host(wl.seed, ids["lora_a"], np.arange(r), K)
+
+    def run(rows):
+        wq, sw = oracle.prepare_weight(synth.weight_host(wl.seed, ids["w_gu"], np.arange(rows), K))
+        b = synth.weight_host(wl.seed, ids["lora_b"], np.arange(rows), r)
+        t0 = time.perf_counter()
+        oracle.lora_merge(wq, sw, a, b, wl.alpha)
+        return time.perf_counter() - t0
+    rows = 64
+    while True:
+        dt = run(rows)
+        if dt >= target_s or rows >= N:
+            break
+        rows = min(N, max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 1.1)))
+    return {"value": 2.0 * rows * K * r / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "rows": rows, "seconds": dt,
+            "sample": f"{rows} of {N} rows of the gate/up weight (K={K}, rank {r}), {dt:.1f} s"}
 
 
 def run_gpu(args):
@@ -643,6 +862,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "lora":
+        return run_lora(args)
     return run_gpu(args)
 
 

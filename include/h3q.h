@@ -142,6 +142,33 @@ h3q_status h3q_ffn_static_scratch(const void* x_bf16, int64_t M, int64_t K,
                                   void* y_bf16, cudaStream_t stream);
 
 /*
+ * LoRA merge into stored int8 weights (h3-rs README, "Speed", "What makes it
+ * fast": LoRAs are merged into the int8 weights at load by dequantizing,
+ * adding and requantizing, so they cost nothing per step). The codes are in the
+ * rotated basis, so the delta is rotated the same way:
+ *   A_rot = A blockdiag(H/16) (the rotation of h3q_prepare_weight, fp32);
+ *   d[n][k] = fma chain over j = 0..r-1 ascending, from 0, of B[n][j] A_rot[j][k];
+ *   w[n][k] = (float)wq[n][k] * sw[n] + alpha * d[n][k]   (fp32, two rounded
+ *             products and one rounded add);
+ *   then each row is requantized: sw[n] = max_k |w[n][k]| / 127,
+ *   wq[n][k] = clamp(rne(w[n][k] / sw[n]), -127, 127) (0 where sw[n] == 0).
+ *   wq [N, K] int8 and sw [N] fp32 are read and overwritten in place.
+ *   lora_a [r, K] fp32 (the LoRA "down" factor, in the model's basis) and
+ *   lora_b [N, r] fp32 (the "up" factor) are read only; alpha is the LoRA
+ *   scale (strength times alpha / rank, as the caller defines it).
+ *   workspace: caller-owned device scratch of at least
+ *   h3q_lora_workspace_size(r, K) bytes, 16-byte aligned (holds A_rot).
+ *   K % 256 == 0, K <= H3Q_MAX_K; 1 <= r <= H3Q_LORA_MAX_RANK; N >= 0
+ *   (N == 0 is a no-op); all pointers 16-byte aligned. Other calls must not
+ *   read or write wq / sw while the merge runs on its stream.
+ */
+#define H3Q_LORA_MAX_RANK 512
+size_t h3q_lora_workspace_size(int64_t r, int64_t K);
+h3q_status h3q_lora_merge(int8_t* wq, float* sw, int64_t N, int64_t K, const float* lora_a,
+                          const float* lora_b, int64_t r, float alpha, void* workspace,
+                          size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Test hook: the same GEMM kernel with the raw int32 accumulators as output.
  *   xq [M, K], wq [N, K] int8; acc [M, N] int32. K % 128 == 0, N % 8 == 0.
  */

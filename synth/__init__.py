@@ -151,13 +151,15 @@ def bias_bf16(seed: int, tensor_id: int, N: int, sigma=SIGMA_BIAS) -> np.ndarray
 # tensor_id = 256 * (block + 1) + local id.
 TID_X, TID_W, TID_BIAS, TID_OUTLIER, TID_WGU, TID_WDOWN = 1, 2, 3, 4, 5, 6
 TID_WQKV, TID_BQKV, TID_WOUT, TID_BOUT, TID_XQKV, TID_XOUT, TID_XFFN = 7, 8, 9, 10, 11, 12, 13
+TID_LORA_A, TID_LORA_B, TID_LORA_A_DOWN, TID_LORA_B_DOWN = 14, 15, 16, 17
 
 
 def tensor_ids(block: int | None = None) -> dict:
     base = 0 if block is None else 256 * (block + 1)
     names = dict(x=TID_X, w=TID_W, bias=TID_BIAS, outlier=TID_OUTLIER, w_gu=TID_WGU, w_down=TID_WDOWN,
                  w_qkv=TID_WQKV, b_qkv=TID_BQKV, w_out=TID_WOUT, b_out=TID_BOUT,
-                 x_qkv=TID_XQKV, x_out=TID_XOUT, x_ffn=TID_XFFN)
+                 x_qkv=TID_XQKV, x_out=TID_XOUT, x_ffn=TID_XFFN, lora_a=TID_LORA_A, lora_b=TID_LORA_B,
+                 lora_a_down=TID_LORA_A_DOWN, lora_b_down=TID_LORA_B_DOWN)
     return {k: base + v for k, v in names.items()}
 
 
@@ -165,10 +167,11 @@ class Workload:
     """Shapes and distributions of one synthetic workload."""
 
     def __init__(self, name, kind, M, K, N=None, F=None, bias=False, n_outliers=0, outlier_factor=1.0,
-                 blocks=1, seed=0):
+                 blocks=1, seed=0, rank=None, alpha=None):
         self.name, self.kind, self.M, self.K, self.N, self.F = name, kind, M, K, N, F
         self.bias, self.n_outliers, self.outlier_factor = bias, n_outliers, outlier_factor
         self.blocks, self.seed = blocks, seed
+        self.rank, self.alpha = rank, alpha
 
     def factors(self, block=None, K=None):
         K = self.K if K is None else K
@@ -179,7 +182,8 @@ class Workload:
 
     def as_dict(self):
         return {k: getattr(self, k) for k in ("name", "kind", "M", "K", "N", "F", "bias", "n_outliers",
-                                                "outlier_factor", "blocks", "seed")}
+                                                "outlier_factor", "blocks", "seed", "rank", "alpha")
+                if getattr(self, k) is not None}
 
 
 def _pct_outliers(K):
@@ -201,6 +205,10 @@ WORKLOADS = {
     # one denoising step's linear sweep: 50 blocks of QKV, out and FFN at 32768 tokens.
     "sweep": Workload("sweep", "sweep", M=32768, K=5376, N=16128, F=14336, bias=True,
                       n_outliers=_pct_outliers(5376), outlier_factor=50.0, blocks=50),
+    # LoRA merge at load into one FFN block's int8 weights (gate/up [28672, 5376]
+    # and down [5376, 14336]): rank-64 factors A [r, K] and B [N, r], both
+    # N(0, 0.02^2), merged with alpha = 1. M is unused (no activations).
+    "lora": Workload("lora", "lora", M=0, K=5376, F=14336, rank=64, alpha=1.0),
 }
 
 

@@ -96,3 +96,27 @@ def test_ffn_rejects_short_workspace_and_bad_shapes():
 
 def test_stalled_wait_rejects_huge_limit():
     assert h3q.lib.h3q_test_stalled_wait(10**12, None) == INV
+
+
+def test_lora_workspace_size():
+    assert h3q.h3q_lora_workspace_size(64, 5376) == 64 * 5376 * 4
+    assert h3q.h3q_lora_workspace_size(0, 5376) == 0
+
+
+def test_lora_merge_rejects():
+    ws = h3q.h3q_lora_workspace_size(8, 512)
+    f = h3q.lib.h3q_lora_merge
+    ok = [FAKE, FAKE, 16, 512, FAKE, FAKE, 8, 1.0, FAKE, ws, None]
+    for i, bad in [(3, 500), (3, 0), (2, -1), (6, 0), (9, ws - 1), (0, None), (4, None), (8, None),
+                   (5, FAKE + 4), (1, FAKE + 8)]:
+        args = list(ok)
+        args[i] = bad
+        assert f(*args) == INV, (i, bad)
+    args = list(ok)
+    args[6] = h3q.H3Q_LORA_MAX_RANK + 1
+    assert f(*args) == h3q.H3Q_ERR_UNSUPPORTED
+    args = list(ok)
+    args[3] = 16384 + 256
+    assert f(*args) == h3q.H3Q_ERR_UNSUPPORTED
+    # N = 0 launches nothing, whatever the pointers
+    assert f(None, None, 0, 512, None, None, 8, 1.0, None, 0, None) == h3q.H3Q_OK

@@ -34,6 +34,8 @@ _SIGS = {
     "h3q_ffn_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "h3q_ffn": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]),
     "h3q_ffn_static_scratch": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _P, _P]),
+    "h3q_lora_workspace_size": (_SZ, [_I64, _I64]),
+    "h3q_lora_merge": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, ctypes.c_float, _P, _SZ, _P]),
     "h3q_gemm_s32": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P]),
     "h3q_get_device_status": (_INT, [_P]),
     "h3q_set_wait_limit_ns": (None, [_U64]),
@@ -119,6 +121,23 @@ def h3q_ffn_static_scratch(x, w_gu, s_gu, w_down, s_down, y, b_gu=None, b_down=N
     _check(lib.h3q_ffn_static_scratch(_ptr(x), M, K, _ptr(w_gu), _ptr(s_gu), _ptr(b_gu), F, _ptr(w_down),
                                       _ptr(s_down), _ptr(b_down), _ptr(y), _stream(stream)),
            "h3q_ffn_static_scratch")
+
+
+H3Q_LORA_MAX_RANK = 512
+
+
+def h3q_lora_workspace_size(r: int, K: int) -> int:
+    return int(lib.h3q_lora_workspace_size(r, K))
+
+
+def h3q_lora_merge(wq, sw, lora_a, lora_b, alpha: float, workspace, stream=None) -> None:
+    """Merge alpha * lora_b @ lora_a (rotated along K) into the int8 weights
+    wq [N, K] / sw [N], in place. lora_a [r, K], lora_b [N, r] fp32."""
+    N, K = wq.shape
+    r = lora_a.shape[0]
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.h3q_lora_merge(_ptr(wq), _ptr(sw), N, K, _ptr(lora_a), _ptr(lora_b), r, float(alpha),
+                              _ptr(workspace), nbytes, _stream(stream)), "h3q_lora_merge")
 
 
 def h3q_gemm_s32(xq, wq, acc, stream=None) -> None:

@@ -11,6 +11,7 @@
 
 #include "h3q.h"
 #include "gemm_sm100.cuh"
+#include "lora.cuh"
 #include "rotquant.cuh"
 
 namespace {
@@ -207,6 +208,25 @@ h3q_status h3q_linear_w8a8(const int8_t* xq, const float* sx, int64_t M, int64_t
   if (epilogue == H3Q_EPI_SWIGLU)
     return launch_gemm<h3q::kEpiSwiGLU>(xq, wq, M, K, N, N / 2, sx, sw, bias_bf16, y_bf16, stream);
   return launch_gemm<h3q::kEpiBF16>(xq, wq, M, K, N, N, sx, sw, bias_bf16, y_bf16, stream);
+}
+
+size_t h3q_lora_workspace_size(int64_t r, int64_t K) {
+  if (r <= 0 || K <= 0) return 0;
+  return size_t(r) * size_t(K) * sizeof(float);
+}
+
+h3q_status h3q_lora_merge(int8_t* wq, float* sw, int64_t N, int64_t K, const float* lora_a, const float* lora_b,
+                          int64_t r, float alpha, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (N < 0 || !valid_k(K) || r < 1) return H3Q_ERR_INVALID_ARG;
+  if (r > H3Q_LORA_MAX_RANK || K > H3Q_MAX_K || N > INT32_MAX) return H3Q_ERR_UNSUPPORTED;
+  if (N == 0) return H3Q_OK;
+  if (!wq || !sw || !lora_a || !lora_b || !workspace) return H3Q_ERR_INVALID_ARG;
+  if (!aligned16(wq) || !aligned16(sw) || !aligned16(lora_a) || !aligned16(lora_b) || !aligned16(workspace))
+    return H3Q_ERR_INVALID_ARG;
+  if (workspace_bytes < h3q_lora_workspace_size(r, K)) return H3Q_ERR_INVALID_ARG;
+  const cudaError_t e = h3q::launch_lora_merge(wq, sw, N, K, lora_a, lora_b, static_cast<int>(r), alpha,
+                                               static_cast<float*>(workspace), stream);
+  return e == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
 }
 
 h3q_status h3q_gemm_s32(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N, int64_t K, int32_t* acc,
