@@ -57,6 +57,13 @@ def _load():
             "orc_lora_merge": (None, [P, P, I64, I64, P, P, I64, F]),
             "orc_f32_to_bf16": (ctypes.c_uint16, [F]),
             "orc_bf16_to_f32": (F, [ctypes.c_uint16]),
+            "orc_e2m1_value": (F, [ctypes.c_uint8]),
+            "orc_e2m1_rne": (ctypes.c_uint8, [F]),
+            "orc_e4m3_value": (F, [ctypes.c_uint8]),
+            "orc_e4m3_rne_sat": (ctypes.c_uint8, [F]),
+            "orc_nvfp4_encode_scale": (F, [P, I64]),
+            "orc_nvfp4_quantize": (None, [P, I64, I64, F, P, P]),
+            "orc_nvfp4_linear": (None, [P, P, F, I64, I64, P, P, F, I64, P, ctypes.c_int, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -250,3 +257,62 @@ def ffn(x_bits, w_gu, s_gu, w_down, s_down, b_gu=None, b_down=None):
     if ovf:
         raise OverflowError(f"{ovf} accumulators outside the int32 range")
     return y, h, hq, sh
+
+
+# ----------------------------------------------------------------------- NVFP4
+def e2m1_value(c: int) -> float:
+    return float(_load().orc_e2m1_value(int(c)))
+
+
+def e2m1_rne(x: float) -> int:
+    return int(_load().orc_e2m1_rne(float(x)))
+
+
+def e4m3_value(c: int) -> float:
+    return float(_load().orc_e4m3_value(int(c)))
+
+
+def e4m3_rne_sat(u: float) -> int:
+    return int(_load().orc_e4m3_rne_sat(float(u)))
+
+
+def nvfp4_encode_scale(x) -> float:
+    """Per-tensor encode scale 2688 / max|x| (x: fp32 values, or bf16 bits as uint16)."""
+    x = _values_f32(x)
+    return float(_load().orc_nvfp4_encode_scale(_p(x), x.size))
+
+
+def _values_f32(x):
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return np.ascontiguousarray((x.astype(np.uint32) << 16).view(np.float32))
+    return _c(x, np.float32)
+
+
+def nvfp4_quantize(x, s_enc=None):
+    """NVFP4 of rows x [rows, K] (fp32, or bf16 bits as uint16). Returns
+    (codes uint8 [rows, K/2], sf uint8 [rows, K/16], s_enc)."""
+    x = _values_f32(x)
+    rows, K = x.shape
+    assert K % 16 == 0
+    if s_enc is None:
+        s_enc = nvfp4_encode_scale(x)
+    codes = np.empty((rows, K // 2), dtype=np.uint8)
+    sf = np.empty((rows, K // 16), dtype=np.uint8)
+    _load().orc_nvfp4_quantize(_p(x), rows, K, float(s_enc), _p(codes), _p(sf))
+    return codes, sf, float(s_enc)
+
+
+def nvfp4_linear(ca, sfa, s_enc_a, cw, sfw, s_enc_w, bias_bits=None, swiglu_epilogue=False):
+    """The NVFP4 layer. Returns (y bf16 bits, acc fp64 [M, N], mag fp64 [M, N])."""
+    ca, sfa, cw, sfw = (_c(a, np.uint8) for a in (ca, sfa, cw, sfw))
+    M, K2 = ca.shape
+    N = cw.shape[0]
+    K = 2 * K2
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    y = np.empty((M, N // 2 if swiglu_epilogue else N), dtype=np.uint16)
+    acc = np.empty((M, N), dtype=np.float64)
+    mag = np.empty((M, N), dtype=np.float64)
+    _load().orc_nvfp4_linear(_p(ca), _p(sfa), float(s_enc_a), M, K, _p(cw), _p(sfw), float(s_enc_w), N, _p(b),
+                             1 if swiglu_epilogue else 0, _p(y), _p(acc), _p(mag))
+    return y, acc, mag

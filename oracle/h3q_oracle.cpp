@@ -328,6 +328,153 @@ void orc_lora_merge(int8_t* q, float* s, int64_t N, int64_t K, const float* lora
   }
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4, the hybrid checkpoints' native Blackwell format for the QKV and
+// FFN-input projections (Minimax_h3_hybrid model card, "Checkpoints" and
+// "Native NVFP4 projection benchmarks"; h3-rs README, model-file table:
+// "NVFP4 (swizzled fp8 block scales)"). The pages do not spell the format out;
+// this follows the public NVFP4 definition: e2m1 elements, one e4m3 scale per
+// 16 consecutive elements along K, one fp32 scale per tensor. No rotation.
+// ---------------------------------------------------------------------------
+
+// e2m1: sign bit 3, two exponent bits (bias 1) and one mantissa bit;
+// magnitudes of codes 0..7: 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+static const float kE2m1Mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+float orc_e2m1_value(uint8_t c) {
+  const float v = kE2m1Mag[c & 7];
+  return (c & 8) ? -v : v;
+}
+
+// Round to the nearest e2m1 magnitude, ties to the even code, saturating at 6;
+// the sign is kept (a negative value that rounds to zero gives -0, code 8).
+uint8_t orc_e2m1_rne(float x) {
+  const float a = std::fabs(x);
+  if (a >= 6.0f) return uint8_t(7 | (std::signbit(x) ? 8 : 0));  // saturate (the search would lose the
+                                                                    // distances of huge values to rounding)
+  int best = 0;
+  float best_d = a;
+  for (int c = 1; c < 8; ++c) {
+    const float d = std::fabs(a - kE2m1Mag[c]);
+    if (d < best_d || (d == best_d && (c & 1) == 0)) {
+      best = c;
+      best_d = d;
+    }
+  }
+  return uint8_t(best | (std::signbit(x) ? 8 : 0));
+}
+
+// e4m3 (OCP FP8 E4M3, as the unsigned block scale): exponent bits 3-6 (bias
+// 7), mantissa bits 0-2; exponent 0 is subnormal (m/8 * 2^-6); code 0x7f is NaN.
+float orc_e4m3_value(uint8_t c) {
+  const int e = (c >> 3) & 15, m = c & 7;
+  const float mag = e == 0 ? std::ldexp(float(m) / 8.0f, -6) : std::ldexp(1.0f + float(m) / 8.0f, e - 7);
+  return (c & 0x80) ? -mag : mag;
+}
+
+// Round a non-negative value to the nearest e4m3 value (ties to the even code),
+// saturating at 448 (the largest finite value).
+uint8_t orc_e4m3_rne_sat(float u) {
+  if (u >= 448.0f) return 0x7e;  // saturate
+  int best = 0;
+  float best_d = std::fabs(u);
+  for (int c = 1; c <= 0x7e; ++c) {
+    const float d = std::fabs(u - orc_e4m3_value(uint8_t(c)));
+    if (d < best_d || (d == best_d && (c & 1) == 0)) {
+      best = c;
+      best_d = d;
+    }
+  }
+  return uint8_t(best);
+}
+
+// The tensor's encode scale: s_enc = RN(2688 / amax) (2688 = 448 * 6: the
+// largest block scale times the largest element), 1 for an all-zero tensor,
+// the largest finite float if the quotient overflows.
+float orc_nvfp4_encode_scale(const float* x, int64_t n) {
+  float amax = 0.0f;
+  for (int64_t i = 0; i < n; ++i) amax = std::fmax(amax, std::fabs(x[i]));
+  if (amax == 0.0f) return 1.0f;
+  const float s = 2688.0f / amax;
+  return std::isinf(s) ? 3.40282347e38f : s;
+}
+
+// Rows [rows, K] (K % 16 == 0) to NVFP4 with encode scale s_enc. Per block of 16
+// consecutive elements of a row, in fp32 and in this order:
+//   S   = e4m3_rne_sat(RN(RN(max|x| / 6) * s_enc))     (the block scale code)
+//   enc = RN(s_enc / value(S))
+//   q   = e2m1_rne(RN(x * enc))                        (0 for every element if S = 0)
+// codes [rows, K/2]: element 2i in the low nibble of byte i; sf [rows, K/16].
+void orc_nvfp4_quantize(const float* x, int64_t rows, int64_t K, float s_enc, uint8_t* codes, uint8_t* sf) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < K / 16; ++b) {
+      const float* v = x + r * K + 16 * b;
+      float bmax = 0.0f;
+      for (int i = 0; i < 16; ++i) bmax = std::fmax(bmax, std::fabs(v[i]));
+      const float t = bmax / 6.0f;
+      const float u = t * s_enc;
+      const uint8_t S = orc_e4m3_rne_sat(u);
+      sf[r * (K / 16) + b] = S;
+      const float Sv = orc_e4m3_value(S);
+      uint8_t q[16];
+      for (int i = 0; i < 16; ++i) {
+        if (S == 0) {
+          q[i] = 0;
+          continue;
+        }
+        const float enc = s_enc / Sv;
+        const float y = v[i] * enc;
+        q[i] = orc_e2m1_rne(y);
+      }
+      for (int i = 0; i < 8; ++i) codes[r * (K / 2) + 8 * b + i] = uint8_t(q[2 * i] | (q[2 * i + 1] << 4));
+    }
+}
+
+// The NVFP4 layer. acc[m][n] = sum over k of e2m1(a) S_a(block of k) e2m1(w)
+// S_w(block of k), summed in fp64 (each block's 16 products are exact, so the
+// sum is exact up to fp64 rounding of the block terms); mag[m][n] = the sum of
+// the block terms' magnitudes (for the error bound of an fp32 accumulation).
+// The output follows the int8 layer's epilogue with the per-tensor factor
+// alpha = RN(1 / RN(s_enc_a * s_enc_w)) in place of sx * sw:
+//   v = RN(RN((float)acc * alpha) + bias);  swiglu: h = silu(v_gate) * v_up.
+// Rows [0, F) of w are the gate and [F, 2F) the up projection when swiglu is set.
+void orc_nvfp4_linear(const uint8_t* ca, const uint8_t* sfa, float s_enc_a, int64_t M, int64_t K,
+                      const uint8_t* cw, const uint8_t* sfw, float s_enc_w, int64_t N, const uint16_t* bias,
+                      int swiglu, uint16_t* y, double* acc, double* mag) {
+  const float alpha = 1.0f / (s_enc_a * s_enc_w);
+  const int64_t KB = K / 16;
+  const int64_t NO = swiglu ? N / 2 : N;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    std::vector<float> v(N);
+    for (int64_t n = 0; n < N; ++n) {
+      double total = 0.0, total_mag = 0.0;
+      for (int64_t b = 0; b < KB; ++b) {
+        double blk = 0.0;
+        for (int i = 0; i < 16; ++i) {
+          const int64_t k = 16 * b + i;
+          const uint8_t qa = (ca[m * (K / 2) + k / 2] >> (4 * (k & 1))) & 15;
+          const uint8_t qw = (cw[n * (K / 2) + k / 2] >> (4 * (k & 1))) & 15;
+          blk += double(orc_e2m1_value(qa)) * double(orc_e2m1_value(qw));
+        }
+        const double term = blk * double(orc_e4m3_value(sfa[m * KB + b])) * double(orc_e4m3_value(sfw[n * KB + b]));
+        total += term;
+        total_mag += std::fabs(term);
+      }
+      if (acc) acc[m * N + n] = total;
+      if (mag) mag[m * N + n] = total_mag;
+      float x = float(total) * alpha;
+      if (bias) x = x + bf16_to_f32(bias[n]);
+      v[n] = x;
+    }
+    for (int64_t j = 0; j < NO; ++j) {
+      const float out = swiglu ? orc_silu_f32(v[j]) * v[NO + j] : v[j];
+      if (y) y[m * NO + j] = f32_to_bf16_rne(out);
+    }
+  }
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();
