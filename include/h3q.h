@@ -169,6 +169,53 @@ h3q_status h3q_lora_merge(int8_t* wq, float* sw, int64_t N, int64_t K, const flo
                           size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * NVFP4 projections. The hybrid checkpoints run the QKV and FFN-input
+ * projections in NVFP4 and keep the output projections INT8 ConvRot
+ * (Minimax_h3_hybrid model card, "Checkpoints" and "Native NVFP4 projection
+ * benchmarks"; h3-rs README, model-file table: "NVFP4 (swizzled fp8 block
+ * scales)"). Format (the public NVFP4 definition; no rotation):
+ *   s_enc = RN(2688 / max|x|) over the whole tensor (1 for an all-zero tensor);
+ *   per 16 consecutive elements of a row, S = e4m3(RN(RN(max|block| / 6) * s_enc))
+ *   (round to nearest even, saturating at 448); codes q = e2m1(RN(x * RN(s_enc /
+ *   S))) (round to nearest even, saturating at 6; 0 where S = 0).
+ * Layouts: codes [rows, K/2] bytes, element 2i in the low nibble of byte i.
+ * Block scales: h3q_nvfp4_sf_bytes(rows, K) bytes in 512-byte atoms of 128 rows
+ * x 4 scales; scale j of row r at byte ((r/128)(K/64) + j/4) * 512 + 16 (r%32)
+ * + 4 ((r%128)/32) + (j%4); rows padded to a multiple of 128 with zero scales.
+ * Tensor scale: a device float[2], [0] = max|x| (as written by the quantizer),
+ * [1] = s_enc.
+ */
+enum { H3Q_DTYPE_BF16 = 0, H3Q_DTYPE_F32 = 1 };
+size_t h3q_nvfp4_sf_bytes(int64_t rows, int64_t K);
+
+/*
+ * x [rows, K] (bf16 activations or fp32 weights, per x_dtype) -> codes, block
+ * scales and the tensor scale, as above. Two launches (tensor max, then the
+ * blocks) and a 4-byte memset of scale[0]. K % 256 == 0, K <= H3Q_MAX_K; all
+ * pointers 16-byte aligned.
+ */
+h3q_status h3q_nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, uint8_t* codes,
+                              uint8_t* sf, float* scale, cudaStream_t stream);
+
+/*
+ * NVFP4 linear: acc[m][n] = sum_k e2m1(x)[m][k] S_x e2m1(w)[n][k] S_w on the
+ * tensor cores (fp32 accumulation); v = RN(RN(acc * alpha) + bias[n]),
+ * alpha = RN(1 / RN(s_enc_x * s_enc_w)); epilogue as h3q_linear_w8a8 (bf16, or
+ * SwiGLU with rows [0, F) of w the gate and [F, 2F) the up projection).
+ *   xc/xsf/x_scale from h3q_nvfp4_quantize of x [M, K]; wc/wsf/w_scale of w [N, K].
+ *   N % 256 == 0 (SwiGLU: N = 2F, F % 128 == 0); K % 256 == 0; M >= 0.
+ * The fp32 accumulation order is the hardware's: results agree with the exact
+ * sum to within fp32 rounding of the K/16 block terms.
+ */
+h3q_status h3q_linear_nvfp4(const uint8_t* xc, const uint8_t* xsf, const float* x_scale, int64_t M, int64_t K,
+                            const uint8_t* wc, const uint8_t* wsf, const float* w_scale, int64_t N,
+                            const void* bias_bf16, int epilogue, void* y_bf16, cudaStream_t stream);
+
+/* Test hook: the same NVFP4 GEMM with the raw fp32 accumulators [M, N] as output. */
+h3q_status h3q_gemm_nvfp4_f32(const uint8_t* xc, const uint8_t* xsf, int64_t M, int64_t K, const uint8_t* wc,
+                              const uint8_t* wsf, int64_t N, float* acc, cudaStream_t stream);
+
+/*
  * Test hook: the same GEMM kernel with the raw int32 accumulators as output.
  *   xq [M, K], wq [N, K] int8; acc [M, N] int32. K % 128 == 0, N % 8 == 0.
  */

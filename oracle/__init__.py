@@ -64,6 +64,7 @@ def _load():
             "orc_nvfp4_encode_scale": (F, [P, I64]),
             "orc_nvfp4_quantize": (None, [P, I64, I64, F, P, P]),
             "orc_nvfp4_linear": (None, [P, P, F, I64, I64, P, P, F, I64, P, ctypes.c_int, P, P, P]),
+            "orc_nvfp4_epilogue": (None, [P, I64, I64, F, F, P, ctypes.c_int, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -316,3 +317,14 @@ def nvfp4_linear(ca, sfa, s_enc_a, cw, sfw, s_enc_w, bias_bits=None, swiglu_epil
     _load().orc_nvfp4_linear(_p(ca), _p(sfa), float(s_enc_a), M, K, _p(cw), _p(sfw), float(s_enc_w), N, _p(b),
                              1 if swiglu_epilogue else 0, _p(y), _p(acc), _p(mag))
     return y, acc, mag
+
+
+def nvfp4_epilogue(acc32, s_enc_a, s_enc_w, bias_bits=None, swiglu_epilogue=False):
+    """The NVFP4 layer's epilogue on given fp32 accumulators [M, N]: bf16 bits."""
+    acc = _c(acc32, np.float32)
+    M, N = acc.shape
+    b = None if bias_bits is None else _c(bias_bits, np.uint16)
+    y = np.empty((M, N // 2 if swiglu_epilogue else N), dtype=np.uint16)
+    _load().orc_nvfp4_epilogue(_p(acc), M, N, float(s_enc_a), float(s_enc_w), _p(b), 1 if swiglu_epilogue else 0,
+                               _p(y))
+    return y

@@ -439,6 +439,24 @@ void orc_nvfp4_quantize(const float* x, int64_t rows, int64_t K, float s_enc, ui
 // alpha = RN(1 / RN(s_enc_a * s_enc_w)) in place of sx * sw:
 //   v = RN(RN((float)acc * alpha) + bias);  swiglu: h = silu(v_gate) * v_up.
 // Rows [0, F) of w are the gate and [F, 2F) the up projection when swiglu is set.
+// The NVFP4 epilogue on given fp32 accumulators acc32 [M, N] (v as above; with
+// swiglu, N = 2F and the output is [M, F]).
+void orc_nvfp4_epilogue(const float* acc32, int64_t M, int64_t N, float s_enc_a, float s_enc_w,
+                        const uint16_t* bias, int swiglu, uint16_t* y) {
+  const float alpha = 1.0f / (s_enc_a * s_enc_w);
+  const int64_t NO = swiglu ? N / 2 : N;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    std::vector<float> v(N);
+    for (int64_t n = 0; n < N; ++n) {
+      float x = acc32[m * N + n] * alpha;
+      if (bias) x = x + bf16_to_f32(bias[n]);
+      v[n] = x;
+    }
+    for (int64_t j = 0; j < NO; ++j) y[m * NO + j] = f32_to_bf16_rne(swiglu ? orc_silu_f32(v[j]) * v[NO + j] : v[j]);
+  }
+}
+
 void orc_nvfp4_linear(const uint8_t* ca, const uint8_t* sfa, float s_enc_a, int64_t M, int64_t K,
                       const uint8_t* cw, const uint8_t* sfw, float s_enc_w, int64_t N, const uint16_t* bias,
                       int swiglu, uint16_t* y, double* acc, double* mag) {

@@ -120,3 +120,21 @@ def test_lora_merge_rejects():
     assert f(*args) == h3q.H3Q_ERR_UNSUPPORTED
     # N = 0 launches nothing, whatever the pointers
     assert f(None, None, 0, 512, None, None, 8, 1.0, None, 0, None) == h3q.H3Q_OK
+
+
+def test_nvfp4_sizes_and_rejects():
+    assert h3q.h3q_nvfp4_sf_bytes(300, 512) == 384 * 32
+    assert h3q.h3q_nvfp4_sf_bytes(128, 5376) == 128 * 336
+    q = h3q.lib.h3q_nvfp4_quantize
+    assert q(FAKE, 0, 4, 500, FAKE, FAKE, FAKE, None) == INV     # K not a multiple of 256
+    assert q(FAKE, 2, 4, 512, FAKE, FAKE, FAKE, None) == INV     # unknown dtype
+    assert q(FAKE, 0, 4, 512, FAKE, FAKE, None, None) == INV     # no scale
+    assert q(FAKE + 8, 0, 4, 512, FAKE, FAKE, FAKE, None) == INV  # misaligned
+    assert q(None, 0, 0, 512, None, None, None, None) == h3q.H3Q_OK
+    lin = h3q.lib.h3q_linear_nvfp4
+    ok = [FAKE, FAKE, FAKE, 4, 512, FAKE, FAKE, FAKE, 512, None, 0, FAKE, None]
+    for i, bad in [(8, 384), (4, 500), (10, 3), (11, None), (0, None), (2, FAKE + 4)]:
+        args = list(ok)
+        args[i] = bad
+        assert lin(*args) == INV, (i, bad)
+    assert h3q.lib.h3q_gemm_nvfp4_f32(FAKE, FAKE, 4, 512, FAKE, FAKE, 100, FAKE, None) == INV

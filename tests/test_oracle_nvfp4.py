@@ -154,3 +154,22 @@ def test_linear_accuracy_and_gate_first_swiglu():
     h2, _, _ = oracle.nvfp4_linear(ca, sfa, ea, np.concatenate([cw[32:], cw[:32]]),
                                    np.concatenate([sfw[32:], sfw[:32]]), ew, swiglu_epilogue=True)
     assert not np.array_equal(h, h2)
+
+
+def test_epilogue_closed_form_and_agreement_with_the_layer():
+    rng = np.random.default_rng(7)
+    # power-of-two tensor scales make alpha exact: v = acc * 2^-16 + bias
+    acc = (rng.integers(-2 ** 20, 2 ** 20, size=(5, 64)) * 0.25).astype(np.float32)
+    bias = torch.from_numpy(rng.standard_normal(64).astype(np.float32)).bfloat16()
+    bb = bias.view(torch.int16).numpy().view(np.uint16)
+    y = oracle.nvfp4_epilogue(acc, 256.0, 256.0, bias_bits=bb)
+    want = (torch.from_numpy(acc.astype(np.float64) * 2.0 ** -16).float() + bias.float()).bfloat16()
+    assert np.array_equal(y, want.view(torch.int16).numpy().view(np.uint16))
+    # the layer's output is its epilogue applied to RN(acc)
+    x = rng.standard_normal((8, 256)).astype(np.float32)
+    w = (rng.standard_normal((32, 256)) * 0.02).astype(np.float32)
+    ca, sfa, ea = oracle.nvfp4_quantize(x)
+    cw, sfw, ew = oracle.nvfp4_quantize(w)
+    for sw in (False, True):
+        y1, a64, _ = oracle.nvfp4_linear(ca, sfa, ea, cw, sfw, ew, swiglu_epilogue=sw)
+        assert np.array_equal(y1, oracle.nvfp4_epilogue(a64.astype(np.float32), ea, ew, swiglu_epilogue=sw))

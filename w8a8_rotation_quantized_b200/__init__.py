@@ -18,6 +18,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "h3q.h")
 
 H3Q_OK, H3Q_ERR_INVALID_ARG, H3Q_ERR_UNSUPPORTED, H3Q_ERR_CUDA, H3Q_ERR_TIMEOUT = range(5)
 H3Q_EPI_NONE, H3Q_EPI_SWIGLU = 0, 1
+H3Q_DTYPE_BF16, H3Q_DTYPE_F32 = 0, 1
 H3Q_MAX_K = 16384
 
 if not os.path.exists(LIB_PATH):
@@ -36,6 +37,10 @@ _SIGS = {
     "h3q_ffn_static_scratch": (_INT, [_P, _I64, _I64, _P, _P, _P, _I64, _P, _P, _P, _P, _P]),
     "h3q_lora_workspace_size": (_SZ, [_I64, _I64]),
     "h3q_lora_merge": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, ctypes.c_float, _P, _SZ, _P]),
+    "h3q_nvfp4_sf_bytes": (_SZ, [_I64, _I64]),
+    "h3q_nvfp4_quantize": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P, _P]),
+    "h3q_linear_nvfp4": (_INT, [_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _INT, _P, _P]),
+    "h3q_gemm_nvfp4_f32": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P]),
     "h3q_gemm_s32": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P]),
     "h3q_get_device_status": (_INT, [_P]),
     "h3q_set_wait_limit_ns": (None, [_U64]),
@@ -138,6 +143,36 @@ def h3q_lora_merge(wq, sw, lora_a, lora_b, alpha: float, workspace, stream=None)
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib.h3q_lora_merge(_ptr(wq), _ptr(sw), N, K, _ptr(lora_a), _ptr(lora_b), r, float(alpha),
                               _ptr(workspace), nbytes, _stream(stream)), "h3q_lora_merge")
+
+
+def h3q_nvfp4_sf_bytes(rows: int, K: int) -> int:
+    return int(lib.h3q_nvfp4_sf_bytes(rows, K))
+
+
+def h3q_nvfp4_quantize(x, codes, sf, scale, stream=None) -> None:
+    """x [rows, K] bf16 or fp32 -> codes uint8 [rows, K/2], sf uint8 [h3q_nvfp4_sf_bytes],
+    scale fp32 [2] (max|x|, s_enc)."""
+    rows, K = x.shape
+    import torch
+    dt = H3Q_DTYPE_BF16 if x.dtype == torch.bfloat16 else H3Q_DTYPE_F32
+    _check(lib.h3q_nvfp4_quantize(_ptr(x), dt, rows, K, _ptr(codes), _ptr(sf), _ptr(scale), _stream(stream)),
+           "h3q_nvfp4_quantize")
+
+
+def h3q_linear_nvfp4(xc, xsf, x_scale, wc, wsf, w_scale, y, bias=None, epilogue=H3Q_EPI_NONE, stream=None) -> None:
+    """y bf16 = NVFP4 linear of x (codes xc [M, K/2]) with w (codes wc [N, K/2])."""
+    M, K2 = xc.shape
+    N = wc.shape[0]
+    _check(lib.h3q_linear_nvfp4(_ptr(xc), _ptr(xsf), _ptr(x_scale), M, 2 * K2, _ptr(wc), _ptr(wsf), _ptr(w_scale), N,
+                                _ptr(bias), int(epilogue), _ptr(y), _stream(stream)), "h3q_linear_nvfp4")
+
+
+def h3q_gemm_nvfp4_f32(xc, xsf, wc, wsf, acc, stream=None) -> None:
+    """acc fp32 [M, N]: the raw NVFP4 accumulators (test hook)."""
+    M, K2 = xc.shape
+    N = wc.shape[0]
+    _check(lib.h3q_gemm_nvfp4_f32(_ptr(xc), _ptr(xsf), M, 2 * K2, _ptr(wc), _ptr(wsf), N, _ptr(acc),
+                                  _stream(stream)), "h3q_gemm_nvfp4_f32")
 
 
 def h3q_gemm_s32(xq, wq, acc, stream=None) -> None:

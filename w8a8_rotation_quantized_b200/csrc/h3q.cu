@@ -6,12 +6,14 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
 #include "h3q.h"
 #include "gemm_sm100.cuh"
 #include "lora.cuh"
+#include "nvfp4.cuh"
 #include "rotquant.cuh"
 
 namespace {
@@ -113,6 +115,56 @@ h3q_status launch_gemm(const int8_t* a, const int8_t* b, int64_t M, int64_t K, i
   const int pairs = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
   const int grid = 2 * pairs;  // clusters of two CTAs
   h3q::gemm_i8_kernel<EPI><<<grid, h3q::kGemmThreads, h3q::kGemmSmem, stream>>>(ta, tb, p);
+  return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+}
+
+// Scale-factor atom array viewed as [bytes / 128, 128] uint8: boxes of 16 rows
+// (2048 bytes = 4 atoms), no swizzle; reads past the end return zeros.
+bool make_tmap_sf(CUtensorMap* map, const void* base, int64_t bytes) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(bytes / 128)};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {128, 16};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+h3q_status launch_gemm_fp4(const uint8_t* a, const uint8_t* a_sf, const float* a_scale, int64_t M, int64_t K,
+                           const uint8_t* b, const uint8_t* b_sf, const float* b_scale, int64_t b_rows,
+                           int64_t N_out, const void* bias, void* out, cudaStream_t stream) {
+  CUtensorMap ta, tb, tsa, tsb;
+  if (!make_tmap_i8(&ta, a, M, K / 2) || !make_tmap_i8(&tb, b, b_rows, K / 2) ||
+      !make_tmap_sf(&tsa, a_sf, h3q::nvfp4_sf_bytes(M, K)) || !make_tmap_sf(&tsb, b_sf, h3q::nvfp4_sf_bytes(b_rows, K)))
+    return H3Q_ERR_CUDA;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(h3q::gemm_fp4_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(h3q::kF4Smem));
+  });
+  if (attr_err != cudaSuccess) return H3Q_ERR_CUDA;
+  h3q::Fp4Params p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N_out);
+  p.K = static_cast<int>(K);
+  p.num_m = static_cast<int>((M + 2 * h3q::kBM - 1) / (2 * h3q::kBM));
+  p.num_n = (EPI == h3q::kEpiSwiGLU) ? static_cast<int>(N_out / 128) : static_cast<int>(N_out / h3q::kBN);
+  p.num_tiles = p.num_m * p.num_n;
+  p.group_m = kGemmGroupRows < p.num_m ? kGemmGroupRows : p.num_m;
+  p.b_row_up = (EPI == h3q::kEpiSwiGLU) ? static_cast<int>(N_out) : 0;
+  p.x_scale = a_scale;
+  p.w_scale = b_scale;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.out = out;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const int sms = sm_count();
+  if (sms <= 0) return H3Q_ERR_CUDA;
+  const int pairs = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
+  h3q::gemm_fp4_kernel<EPI><<<2 * pairs, h3q::kGemmThreads, h3q::kF4Smem, stream>>>(ta, tb, tsa, tsb, p);
   return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
 }
 
@@ -227,6 +279,75 @@ h3q_status h3q_lora_merge(int8_t* wq, float* sw, int64_t N, int64_t K, const flo
   const cudaError_t e = h3q::launch_lora_merge(wq, sw, N, K, lora_a, lora_b, static_cast<int>(r), alpha,
                                                static_cast<float*>(workspace), stream);
   return e == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+}
+
+size_t h3q_nvfp4_sf_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K <= 0 || K % 64 != 0) return 0;
+  return static_cast<size_t>(h3q::nvfp4_sf_bytes(rows, K));
+}
+
+h3q_status h3q_nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t K, uint8_t* codes, uint8_t* sf,
+                              float* scale, cudaStream_t stream) {
+  if (rows < 0 || !valid_k(K) || (x_dtype != H3Q_DTYPE_BF16 && x_dtype != H3Q_DTYPE_F32)) return H3Q_ERR_INVALID_ARG;
+  if (K > H3Q_MAX_K || rows > INT32_MAX) return H3Q_ERR_UNSUPPORTED;
+  if (rows == 0) return H3Q_OK;
+  if (!x || !codes || !sf || !scale || !aligned16(x) || !aligned16(codes) || !aligned16(sf) || !aligned16(scale))
+    return H3Q_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return H3Q_ERR_CUDA;
+  if (cudaMemsetAsync(scale, 0, sizeof(uint32_t), stream) != cudaSuccess) return H3Q_ERR_CUDA;
+  const int64_t n16 = rows * K / 16;
+  const int64_t rows_pad = (rows + 127) / 128 * 128;
+  const int64_t total = rows_pad * (K / 16);
+  const unsigned g1 = static_cast<unsigned>(std::min<int64_t>((n16 + 255) / 256, int64_t(sms) * 8));
+  const unsigned g2 = static_cast<unsigned>(std::min<int64_t>((total + 255) / 256, int64_t(sms) * 16));
+  uint32_t* amax = reinterpret_cast<uint32_t*>(scale);
+  if (x_dtype == H3Q_DTYPE_BF16) {
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    h3q::nvfp4_amax_kernel<__nv_bfloat16><<<g1, 256, 0, stream>>>(xb, n16, amax);
+    h3q::nvfp4_quantize_kernel<__nv_bfloat16><<<g2, 256, 0, stream>>>(xb, rows, rows_pad, static_cast<int>(K), scale,
+                                                                     codes, sf);
+  } else {
+    const float* xf = static_cast<const float*>(x);
+    h3q::nvfp4_amax_kernel<float><<<g1, 256, 0, stream>>>(xf, n16, amax);
+    h3q::nvfp4_quantize_kernel<float><<<g2, 256, 0, stream>>>(xf, rows, rows_pad, static_cast<int>(K), scale, codes,
+                                                             sf);
+  }
+  return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+}
+
+static h3q_status check_fp4_args(const uint8_t* xc, const uint8_t* xsf, const float* x_scale, int64_t M, int64_t K,
+                                 const uint8_t* wc, const uint8_t* wsf, const float* w_scale, int64_t N) {
+  if (M < 0 || !valid_k(K) || N <= 0 || N % 256 != 0) return H3Q_ERR_INVALID_ARG;
+  if (K > H3Q_MAX_K || M > INT32_MAX - 256 || N > INT32_MAX - 512) return H3Q_ERR_UNSUPPORTED;
+  if (M == 0) return H3Q_OK;
+  if (!xc || !xsf || !x_scale || !wc || !wsf || !w_scale) return H3Q_ERR_INVALID_ARG;
+  if (!aligned16(xc) || !aligned16(xsf) || !aligned16(wc) || !aligned16(wsf) ||
+      (reinterpret_cast<uintptr_t>(x_scale) & 7u) || (reinterpret_cast<uintptr_t>(w_scale) & 7u))
+    return H3Q_ERR_INVALID_ARG;
+  return H3Q_OK;
+}
+
+h3q_status h3q_linear_nvfp4(const uint8_t* xc, const uint8_t* xsf, const float* x_scale, int64_t M, int64_t K,
+                            const uint8_t* wc, const uint8_t* wsf, const float* w_scale, int64_t N,
+                            const void* bias_bf16, int epilogue, void* y_bf16, cudaStream_t stream) {
+  if (epilogue != H3Q_EPI_NONE && epilogue != H3Q_EPI_SWIGLU) return H3Q_ERR_INVALID_ARG;
+  const h3q_status st = check_fp4_args(xc, xsf, x_scale, M, K, wc, wsf, w_scale, N);
+  if (st != H3Q_OK || M == 0) return st;
+  if (!y_bf16 || !aligned16(y_bf16) || (bias_bf16 && !aligned16(bias_bf16))) return H3Q_ERR_INVALID_ARG;
+  if (epilogue == H3Q_EPI_SWIGLU)
+    return launch_gemm_fp4<h3q::kEpiSwiGLU>(xc, xsf, x_scale, M, K, wc, wsf, w_scale, N, N / 2, bias_bf16, y_bf16,
+                                            stream);
+  return launch_gemm_fp4<h3q::kEpiBF16>(xc, xsf, x_scale, M, K, wc, wsf, w_scale, N, N, bias_bf16, y_bf16, stream);
+}
+
+h3q_status h3q_gemm_nvfp4_f32(const uint8_t* xc, const uint8_t* xsf, int64_t M, int64_t K, const uint8_t* wc,
+                              const uint8_t* wsf, int64_t N, float* acc, cudaStream_t stream) {
+  static const float kUnused[2] = {0.0f, 0.0f};  // the raw-accumulator epilogue reads no tensor scale
+  const h3q_status st = check_fp4_args(xc, xsf, kUnused, M, K, wc, wsf, kUnused, N);
+  if (st != H3Q_OK || M == 0) return st;
+  if (!acc || !aligned16(acc)) return H3Q_ERR_INVALID_ARG;
+  return launch_gemm_fp4<h3q::kEpiS32>(xc, xsf, nullptr, M, K, wc, wsf, nullptr, N, N, nullptr, acc, stream);
 }
 
 h3q_status h3q_gemm_s32(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N, int64_t K, int32_t* acc,
