@@ -22,6 +22,11 @@ Workload lora: merging a rank-64 LoRA at load into one FFN block's int8
 weights (gate/up [28672, 5376] and down [5376, 14336]); value in fp32 TFLOP/s of
 the merge's low-rank product, bound by the fp32 FMA pipe.
 
+Workload nvfp4: the hybrid checkpoints' four linear operations of one block at
+16000 tokens (QKV and FFN input in NVFP4, attention output and FFN output in
+INT8 ConvRot, each with the quantization of its input), next to the same four
+operations all in INT8 ConvRot; value in TOPS of the four GEMMs.
+
 Multi-GPU (torchrun): every rank runs its own batch with replicated weights
 (the rows are independent; there is no data-path collective). Times are the
 max over ranks; the value is the work of all ranks over that time.
@@ -52,7 +57,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="h3q", choices=["h3q", "reference"])
-    ap.add_argument("--workload", default="ffn", choices=["ffn", "qkv", "out", "tiny", "sweep", "lora"])
+    ap.add_argument("--workload", default="ffn", choices=["ffn", "qkv", "out", "tiny", "sweep", "lora", "nvfp4"])
     ap.add_argument("--M", type=int, default=None, help="tokens per GPU (default: the workload's)")
     ap.add_argument("--F", type=int, default=None, help="FFN width (default 14336)")
     ap.add_argument("--kernel-reps", type=int, default=10)
@@ -243,6 +248,22 @@ def run_reference(args):
     import oracle
     import synth
 
+    if args.workload == "nvfp4":
+        per_step = 60.0 / max(1, args.steps + args.warmup)
+        for _ in range(args.warmup):
+            oracle_nvfp4_rate(per_step)
+        vals = [oracle_nvfp4_rate(per_step) for _ in range(args.steps)]
+        secs = sum(v["seconds"] for v in vals)
+        value = sum(v["value"] * v["seconds"] for v in vals) / secs
+        line = {"impl": "reference", "metric": "hybrid NVFP4/INT8 linear TOPS", "value": value, "unit": "TOPS",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4+i8",
+                "data": "synthetic", "config": {"workload": "NVFP4 QKV projection, sampled rows"},
+                "cpu_baseline": {"value": value, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+                                 "sample": vals[-1]["sample"]},
+                "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
     if args.workload == "lora":
         per_step = 60.0 / max(1, args.steps + args.warmup)
         for _ in range(args.warmup):
@@ -575,6 +596,190 @@ def run_lora(args):
     return 0
 
 
+NVFP4_OPS = [  # (name, K, N, SwiGLU, NVFP4 in the hybrid)
+    ("qkv", 5376, 16128, False, True),
+    ("attn_out", 5376, 5376, False, False),
+    ("ffn_in", 5376, 28672, True, True),
+    ("ffn_out", 14336, 5376, False, False),
+]
+
+
+def run_nvfp4(args):
+    """The hybrid block's four linear operations (NVFP4 for QKV and FFN input,
+    INT8 ConvRot for the output projections) against all-INT8 ConvRot."""
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import w8a8_rotation_quantized_b200 as h3q
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    M = args.M or 16000
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    ids = synth.tensor_ids()
+    K0 = 5376
+    factors = torch.from_numpy(synth.column_factors(K0, synth.outlier_columns(0, ids["outlier"], K0, 54), 50.0)).to(dev)
+    row0, _ = shard_rows(rank, world, M)
+    x = {}
+    for name, tid in (("qkv", ids["x_qkv"]), ("attn_out", ids["x_out"]), ("ffn_in", ids["x_ffn"])):
+        t = torch.empty((M, K0), dtype=torch.bfloat16, device=dev)
+        synth.fill_device(0, tid, row0, M, K0, t.data_ptr(), sp, factors_ptr=factors.data_ptr(), bf16=True)
+        x[name] = t
+    ops = {}
+    for name, K, N, swiglu, fp4 in NVFP4_OPS:
+        tid = {"qkv": ids["w_qkv"], "attn_out": ids["w_out"], "ffn_in": ids["w_gu"], "ffn_out": ids["w_down"]}[name]
+        w = torch.empty((N, K), dtype=torch.float32, device=dev)
+        synth.fill_device(0, tid, 0, N, K, w.data_ptr(), sp, scale=float(synth.SIGMA_W), bf16=False)
+        o = dict(K=K, N=N, swiglu=swiglu, fp4=fp4, epi=h3q.H3Q_EPI_SWIGLU if swiglu else h3q.H3Q_EPI_NONE)
+        o["wq"] = torch.empty((N, K), dtype=torch.int8, device=dev)
+        o["sw"] = torch.empty(N, dtype=torch.float32, device=dev)
+        h3q.h3q_prepare_weight(w, o["wq"], o["sw"])
+        if True:  # NVFP4 weights for every op: the hybrid uses two, the per-op table all four
+            o["wc"] = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+            o["wsf"] = torch.empty(h3q.h3q_nvfp4_sf_bytes(N, K), dtype=torch.uint8, device=dev)
+            o["ws"] = torch.empty(2, dtype=torch.float32, device=dev)
+            h3q.h3q_nvfp4_quantize(w, o["wc"], o["wsf"], o["ws"])
+            o["xc"] = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+            o["xsf"] = torch.empty(h3q.h3q_nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=dev)
+            o["xs"] = torch.empty(2, dtype=torch.float32, device=dev)
+        del w
+        o["xq"] = torch.empty((M, K), dtype=torch.int8, device=dev)
+        o["sx"] = torch.empty(M, dtype=torch.float32, device=dev)
+        o["y"] = torch.empty((M, N // 2 if swiglu else N), dtype=torch.bfloat16, device=dev)
+        ops[name] = o
+    x["ffn_out"] = ops["ffn_in"]["y"]  # h, produced by the FFN input projection within the step
+
+    def run_op(name, use_fp4):
+        o = ops[name]
+        if use_fp4:
+            h3q.h3q_nvfp4_quantize(x[name], o["xc"], o["xsf"], o["xs"])
+            h3q.h3q_linear_nvfp4(o["xc"], o["xsf"], o["xs"], o["wc"], o["wsf"], o["ws"], o["y"], epilogue=o["epi"])
+        else:
+            h3q.h3q_rotate_quant(x[name], o["xq"], o["sx"])
+            h3q.h3q_linear_w8a8(o["xq"], o["sx"], o["wq"], o["sw"], o["y"], epilogue=o["epi"])
+
+    def step(hybrid=True):
+        for name, _, _, _, fp4 in NVFP4_OPS:
+            run_op(name, hybrid and fp4)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, n):
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for i in range(n):
+            flush.fill_(i & 0xFF)
+            st[i].record(stream)
+            fn()
+            en[i].record(stream)
+        barrier()
+        return sum(a.elapsed_time(b) for a, b in zip(st, en))
+
+    steps = max(1, min(args.steps, 50))
+    for _ in range(args.warmup):
+        step(True)
+        step(False)
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.5)
+    t_host0 = time.time()
+    total_ms = max_over_ranks(timed(lambda: step(True), steps), dev)
+    clk = clocks.stop(t_host0, time.time())
+    int8_ms = max_over_ranks(timed(lambda: step(False), steps), dev) / steps
+    st = h3q.h3q_get_device_status()
+    if st != h3q.H3Q_OK:
+        raise RuntimeError(f"device status after the timed region: {h3q.h3q_status_string(st)}")
+    per_op = {}
+    for name, K, N, swiglu, fp4 in NVFP4_OPS:
+        reps = max(3, args.kernel_reps)
+        t8 = max_over_ranks(timed(lambda: run_op(name, False), reps), dev) / reps
+        t4 = max_over_ranks(timed(lambda: run_op(name, True), reps), dev) / reps
+        per_op[name] = {"int8_convrot_ms": t8, "nvfp4_ms": t4, "change": t4 / t8 - 1.0, "nvfp4_in_hybrid": fp4}
+    o = ops["ffn_in"]
+    reps = max(3, args.kernel_reps)
+    dom_ms = max_over_ranks(timed(lambda: h3q.h3q_linear_nvfp4(o["xc"], o["xsf"], o["xs"], o["wc"], o["wsf"], o["ws"],
+                                                                o["y"], epilogue=o["epi"]), reps), dev) / reps
+    if rank == 0:
+        ms = total_ms / steps
+        flops = sum(2.0 * M * N * K for _, K, N, _, _ in NVFP4_OPS)
+        peaks, peak_src = measured_peaks()
+        fp4_peak = 4.0 * peaks["bf16_tflops"]
+        achieved = 2.0 * M * 28672 * 5376 / (dom_ms * 1e-3) / 1e12
+        line = {
+            "metric": "hybrid NVFP4/INT8 linear TOPS", "value": job_tops(flops, world, ms), "unit": "TOPS",
+            "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp4+i8", "data": "synthetic",
+            "config": {"workload": f"one block's four linear operations at M={M}: QKV {K0}->16128 and FFN input "
+                                   f"{K0}->2x14336+SwiGLU in NVFP4, attention output {K0}->{K0} and FFN output "
+                                   f"14336->{K0} in INT8 ConvRot, each with its input's quantization",
+                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+                       "parallelism": f"replicas x{world}"},
+            "all_int8_convrot_ms_per_step": int8_ms,
+            "hybrid_vs_int8": int8_ms / ms,
+            "per_op_ms": per_op,
+            "roofline": {"bound": "tensor", "kernel": "gemm_fp4_kernel<SwiGLU> (FFN input)", "achieved": achieved,
+                         "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                         "traffic": traffic_from_profile("gemm_fp4_swiglu_ffn_in"),
+                         "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 "
+                                        "(dense fp4/bf16 nominal ratio 9/2.25)"},
+            "gpu_launches": 10 * steps,
+            "clocks": clk,
+            "e2e": None,
+        }
+        if not args.no_cpu_baseline:
+            try:
+                line["cpu_baseline"] = oracle_nvfp4_rate(args.cpu_seconds)
+            except Exception as exc:
+                line["cpu_baseline"] = {"value": None, "error": repr(exc)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def oracle_nvfp4_rate(target_s):
+    """The oracle's NVFP4 layer on a bounded sample of rows of the QKV projection
+    (full weight); GEMM flops per second."""
+    import numpy as np
+
+    import oracle
+    import synth
+    ids = synth.tensor_ids()
+    K, N = 5376, 16128
+    cw, sfw, ew = oracle.nvfp4_quantize(synth.weight_host(0, ids["w_qkv"], np.arange(N), K))
+
+    def run(rows):
+        ca, sfa, ea = oracle.nvfp4_quantize(synth.activation_host(0, ids["x_qkv"], np.arange(rows), K))
+        t0 = time.perf_counter()
+        oracle.nvfp4_linear(ca, sfa, ea, cw, sfw, ew)
+        return time.perf_counter() - t0
+    rows = 2
+    while True:
+        dt = run(rows)
+        if dt >= target_s or rows >= 4096:
+            break
+        rows = min(4096, max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 1.1)))
+    return {"value": 2.0 * rows * N * K / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "rows": rows, "seconds": dt,
+            "sample": f"{rows} token rows of the QKV projection in NVFP4 (full weight), {dt:.1f} s"}
+
+
 def oracle_lora_rate(target_s, steps=None):
     """The oracle's LoRA merge on a bounded sample of the gate/up weight's rows
     (full K and rank); flops of the low-rank product per second."""
@@ -864,6 +1069,8 @@ def main():
         return run_reference(args)
     if args.workload == "lora":
         return run_lora(args)
+    if args.workload == "nvfp4":
+        return run_nvfp4(args)
     return run_gpu(args)
 
 
