@@ -65,6 +65,7 @@ def _load():
             "orc_nvfp4_quantize": (None, [P, I64, I64, F, P, P]),
             "orc_nvfp4_linear": (None, [P, P, F, I64, I64, P, P, F, I64, P, ctypes.c_int, P, P, P]),
             "orc_nvfp4_epilogue": (None, [P, I64, I64, F, F, P, ctypes.c_int, P]),
+            "orc_attention_int8": (None, [P, P, P, I64, I64, I64, I64, P, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -328,3 +329,20 @@ def nvfp4_epilogue(acc32, s_enc_a, s_enc_w, bias_bits=None, swiglu_epilogue=Fals
     _load().orc_nvfp4_epilogue(_p(acc), M, N, float(s_enc_a), float(s_enc_w), _p(b), 1 if swiglu_epilogue else 0,
                                _p(y))
     return y
+
+
+# ------------------------------------------------------------ int8 attention
+def attention_int8(q_bits, k_bits, v_bits, H, D=128):
+    """int8 Q.K^T / softmax / P.V per head. q, k, v: bf16 bits [S, ld], head h at
+    columns h*D .. h*D+D-1. Returns (o float64 [S, H*D], qq int8 [H, S, D],
+    qs fp32 [H, S], kq, ks)."""
+    q, k, v = (_c(a, np.uint16) for a in (q_bits, k_bits, v_bits))
+    assert q.shape == k.shape == v.shape and q.shape[1] >= H * D
+    S, ld = q.shape
+    qq = np.empty((H, S, D), dtype=np.int8)
+    kq = np.empty((H, S, D), dtype=np.int8)
+    qs = np.empty((H, S), dtype=np.float32)
+    ks = np.empty((H, S), dtype=np.float32)
+    o = np.empty((S, H * D), dtype=np.float64)
+    _load().orc_attention_int8(_p(q), _p(k), _p(v), S, D, H, ld, _p(qq), _p(qs), _p(kq), _p(ks), _p(o))
+    return o, qq, qs, kq, ks

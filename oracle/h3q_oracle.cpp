@@ -493,6 +493,52 @@ void orc_nvfp4_linear(const uint8_t* ca, const uint8_t* sfa, float s_enc_a, int6
   }
 }
 
+// ---------------------------------------------------------------------------
+// int8 attention (h3-rs README, "What makes it fast": the DiT attention runs an
+// int8 Q.K^T / 16-bit P.V flash kernel). Per head h (columns h*D .. h*D+D-1 of
+// the [S, ld] q, k, v matrices, bf16 bit patterns):
+//   Q and K rows (one token of one head) are quantized like weight rows
+//   (steps 3-4: s = max|x| / 127 in fp32, codes clamp(rne(x / s)));
+//   s_ij = (sum_d Qq_id Kq_jd) * qs_i * ks_j / sqrt(D)   (exact integer dot product)
+//   O_i  = sum_j softmax_j(s_i)_j V_j                      (float64)
+// qq, kq [H, S, D] int8 and qs, ks [H, S]; o [S, H*D] float64.
+// ---------------------------------------------------------------------------
+void orc_attention_int8(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S, int64_t D, int64_t H,
+                        int64_t ld, int8_t* qq, float* qs, int8_t* kq, float* ks, double* o) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < H * S; ++t) {
+    const int64_t h = t / S, i = t % S;
+    std::vector<float> row(D);
+    for (int64_t d = 0; d < D; ++d) row[d] = bf16_to_f32(q[i * ld + h * D + d]);
+    quantize_row(row.data(), D, qq + t * D, qs + t);
+    for (int64_t d = 0; d < D; ++d) row[d] = bf16_to_f32(k[i * ld + h * D + d]);
+    quantize_row(row.data(), D, kq + t * D, ks + t);
+  }
+  const double inv_sqrt_d = 1.0 / std::sqrt(double(D));
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < H * S; ++t) {
+    const int64_t h = t / S, i = t % S;
+    std::vector<double> sc(S);
+    double mx = -INFINITY;
+    for (int64_t j = 0; j < S; ++j) {
+      int64_t dot = 0;
+      for (int64_t d = 0; d < D; ++d) dot += int64_t(qq[t * D + d]) * int64_t(kq[(h * S + j) * D + d]);
+      sc[j] = double(dot) * double(qs[t]) * double(ks[h * S + j]) * inv_sqrt_d;
+      mx = std::fmax(mx, sc[j]);
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < S; ++j) {
+      sc[j] = std::exp(sc[j] - mx);
+      l += sc[j];
+    }
+    for (int64_t d = 0; d < D; ++d) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < S; ++j) acc += sc[j] * double(bf16_to_f32(v[j * ld + h * D + d]));
+      o[i * H * D + h * D + d] = acc / l;
+    }
+  }
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();
