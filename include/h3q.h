@@ -216,6 +216,32 @@ h3q_status h3q_gemm_nvfp4_f32(const uint8_t* xc, const uint8_t* xsf, int64_t M, 
                               const uint8_t* wsf, int64_t N, float* acc, cudaStream_t stream);
 
 /*
+ * int8 attention for the DiT blocks (h3-rs README, "What makes it fast": an
+ * int8 Q.K^T / 16-bit P.V flash kernel). Head dim 128; head h of q, k, v and out
+ * is columns h*128 .. h*128+127 of a row-major [S, ld] bf16 matrix (q, k and v
+ * may be column slices of one QKV projection output).
+ *   Q and K rows (one token of one head) are quantized like weight rows:
+ *   s = max|x| / 127 (fp32), codes clamp(rne(x / s));
+ *   s_ij = (sum_d Qq_id Kq_jd) qs_i ks_j / sqrt(128); O_i = softmax_j(s_i) V;
+ *   P is rounded to bf16 and P.V accumulated in fp32 (the hardware's order);
+ *   out = bf16(O).
+ * workspace: h3q_attention_workspace_size(S, H) bytes, 256-byte aligned (codes,
+ * scales and V transposed per head). S % 8 == 0, ld % 8 == 0, ld >= 128 H,
+ * ld_out likewise; pointers 16-byte aligned.
+ */
+size_t h3q_attention_workspace_size(int64_t S, int64_t H);
+h3q_status h3q_attention_int8(const void* q, const void* k, const void* v, int64_t S, int64_t H, int64_t ld,
+                              void* out, int64_t ld_out, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
+/*
+ * The attention's input pass on its own (test hook and building block): qq, kq
+ * int8 [H, S, 128], qs, ks fp32 [H, S], vt bf16 [H*128, S] (V^T per head).
+ */
+h3q_status h3q_attention_prep(const void* q, const void* k, const void* v, int64_t S, int64_t H, int64_t ld,
+                              int8_t* qq, float* qs, int8_t* kq, float* ks, void* vt, cudaStream_t stream);
+
+/*
  * Test hook: the same GEMM kernel with the raw int32 accumulators as output.
  *   xq [M, K], wq [N, K] int8; acc [M, N] int32. K % 128 == 0, N % 8 == 0.
  */

@@ -65,7 +65,7 @@ def _load():
             "orc_nvfp4_quantize": (None, [P, I64, I64, F, P, P]),
             "orc_nvfp4_linear": (None, [P, P, F, I64, I64, P, P, F, I64, P, ctypes.c_int, P, P, P]),
             "orc_nvfp4_epilogue": (None, [P, I64, I64, F, F, P, ctypes.c_int, P]),
-            "orc_attention_int8": (None, [P, P, P, I64, I64, I64, I64, P, P, P, P, P]),
+            "orc_attention_int8": (None, [P, P, P, I64, I64, I64, I64, P, P, P, P, P, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -332,10 +332,10 @@ def nvfp4_epilogue(acc32, s_enc_a, s_enc_w, bias_bits=None, swiglu_epilogue=Fals
 
 
 # ------------------------------------------------------------ int8 attention
-def attention_int8(q_bits, k_bits, v_bits, H, D=128):
+def attention_int8(q_bits, k_bits, v_bits, H, D=128, rows=None):
     """int8 Q.K^T / softmax / P.V per head. q, k, v: bf16 bits [S, ld], head h at
-    columns h*D .. h*D+D-1. Returns (o float64 [S, H*D], qq int8 [H, S, D],
-    qs fp32 [H, S], kq, ks)."""
+    columns h*D .. h*D+D-1. Returns (o float64 [n, H*D] for the query rows
+    `rows` (all rows if None), qq int8 [H, S, D], qs fp32 [H, S], kq, ks)."""
     q, k, v = (_c(a, np.uint16) for a in (q_bits, k_bits, v_bits))
     assert q.shape == k.shape == v.shape and q.shape[1] >= H * D
     S, ld = q.shape
@@ -343,6 +343,8 @@ def attention_int8(q_bits, k_bits, v_bits, H, D=128):
     kq = np.empty((H, S, D), dtype=np.int8)
     qs = np.empty((H, S), dtype=np.float32)
     ks = np.empty((H, S), dtype=np.float32)
-    o = np.empty((S, H * D), dtype=np.float64)
-    _load().orc_attention_int8(_p(q), _p(k), _p(v), S, D, H, ld, _p(qq), _p(qs), _p(kq), _p(ks), _p(o))
+    r = None if rows is None else _c(rows, np.int64)
+    n = S if r is None else r.size
+    o = np.empty((n, H * D), dtype=np.float64)
+    _load().orc_attention_int8(_p(q), _p(k), _p(v), S, D, H, ld, _p(qq), _p(qs), _p(kq), _p(ks), _p(r), n, _p(o))
     return o, qq, qs, kq, ks

@@ -501,10 +501,13 @@ void orc_nvfp4_linear(const uint8_t* ca, const uint8_t* sfa, float s_enc_a, int6
 //   (steps 3-4: s = max|x| / 127 in fp32, codes clamp(rne(x / s)));
 //   s_ij = (sum_d Qq_id Kq_jd) * qs_i * ks_j / sqrt(D)   (exact integer dot product)
 //   O_i  = sum_j softmax_j(s_i)_j V_j                      (float64)
-// qq, kq [H, S, D] int8 and qs, ks [H, S]; o [S, H*D] float64.
+// qq, kq [H, S, D] int8 and qs, ks [H, S]; o [n, H*D] float64 for the query
+// rows rows[0..n) (all S rows in order when rows is null).
 // ---------------------------------------------------------------------------
 void orc_attention_int8(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S, int64_t D, int64_t H,
-                        int64_t ld, int8_t* qq, float* qs, int8_t* kq, float* ks, double* o) {
+                        int64_t ld, int8_t* qq, float* qs, int8_t* kq, float* ks, const int64_t* rows, int64_t n,
+                        double* o) {
+  if (!rows) n = S;
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < H * S; ++t) {
     const int64_t h = t / S, i = t % S;
@@ -516,8 +519,10 @@ void orc_attention_int8(const uint16_t* q, const uint16_t* k, const uint16_t* v,
   }
   const double inv_sqrt_d = 1.0 / std::sqrt(double(D));
 #pragma omp parallel for schedule(dynamic, 1)
-  for (int64_t t = 0; t < H * S; ++t) {
-    const int64_t h = t / S, i = t % S;
+  for (int64_t u = 0; u < H * n; ++u) {
+    const int64_t h = u / n, r = u % n;
+    const int64_t i = rows ? rows[r] : r;
+    const int64_t t = h * S + i;
     std::vector<double> sc(S);
     double mx = -INFINITY;
     for (int64_t j = 0; j < S; ++j) {
@@ -534,7 +539,7 @@ void orc_attention_int8(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     for (int64_t d = 0; d < D; ++d) {
       double acc = 0.0;
       for (int64_t j = 0; j < S; ++j) acc += sc[j] * double(bf16_to_f32(v[j * ld + h * D + d]));
-      o[i * H * D + h * D + d] = acc / l;
+      o[r * H * D + h * D + d] = acc / l;
     }
   }
 }

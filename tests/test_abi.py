@@ -138,3 +138,16 @@ def test_nvfp4_sizes_and_rejects():
         args[i] = bad
         assert lin(*args) == INV, (i, bad)
     assert h3q.lib.h3q_gemm_nvfp4_f32(FAKE, FAKE, 4, 512, FAKE, FAKE, 100, FAKE, None) == INV
+
+
+def test_attention_rejects():
+    f = h3q.lib.h3q_attention_int8
+    ws = h3q.h3q_attention_workspace_size(64, 2)
+    assert ws >= 2 * 64 * 128 * 4 + 2 * 2 * 64 * 4
+    ok = [FAKE, FAKE, FAKE, 64, 2, 256, FAKE, 256, FAKE, ws, None]
+    for i, bad in [(3, 60), (4, 0), (5, 200), (5, 260), (7, 100), (9, ws - 1), (8, FAKE + 16), (0, None),
+                   (6, FAKE + 8)]:
+        args = list(ok)
+        args[i] = bad
+        assert f(*args) == INV, (i, bad)
+    assert f(None, None, None, 0, 2, 256, None, 256, None, 0, None) == h3q.H3Q_OK

@@ -41,6 +41,9 @@ _SIGS = {
     "h3q_nvfp4_quantize": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P, _P]),
     "h3q_linear_nvfp4": (_INT, [_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _INT, _P, _P]),
     "h3q_gemm_nvfp4_f32": (_INT, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P]),
+    "h3q_attention_workspace_size": (_SZ, [_I64, _I64]),
+    "h3q_attention_int8": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _SZ, _P]),
+    "h3q_attention_prep": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P]),
     "h3q_gemm_s32": (_INT, [_P, _P, _I64, _I64, _I64, _P, _P]),
     "h3q_get_device_status": (_INT, [_P]),
     "h3q_set_wait_limit_ns": (None, [_U64]),
@@ -173,6 +176,30 @@ def h3q_gemm_nvfp4_f32(xc, xsf, wc, wsf, acc, stream=None) -> None:
     N = wc.shape[0]
     _check(lib.h3q_gemm_nvfp4_f32(_ptr(xc), _ptr(xsf), M, 2 * K2, _ptr(wc), _ptr(wsf), N, _ptr(acc),
                                   _stream(stream)), "h3q_gemm_nvfp4_f32")
+
+
+def h3q_attention_workspace_size(S: int, H: int) -> int:
+    return int(lib.h3q_attention_workspace_size(S, H))
+
+
+def _ld(t):
+    return t.stride(0)
+
+
+def h3q_attention_int8(q, k, v, H, out, workspace, stream=None) -> None:
+    """out [S, >= 128 H] bf16 = int8 attention of q, k, v ([S, ld] bf16 views, head h
+    at columns h*128; q, k, v may be column slices of one matrix)."""
+    S = q.shape[0]
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.h3q_attention_int8(_ptr(q), _ptr(k), _ptr(v), S, H, _ld(q), _ptr(out), _ld(out), _ptr(workspace),
+                                  nbytes, _stream(stream)), "h3q_attention_int8")
+
+
+def h3q_attention_prep(q, k, v, H, qq, qs, kq, ks, vt, stream=None) -> None:
+    """The attention's input pass: int8 Q/K codes and scales per head, V^T per head."""
+    S = q.shape[0]
+    _check(lib.h3q_attention_prep(_ptr(q), _ptr(k), _ptr(v), S, H, _ld(q), _ptr(qq), _ptr(qs), _ptr(kq), _ptr(ks),
+                                  _ptr(vt), _stream(stream)), "h3q_attention_prep")
 
 
 def h3q_gemm_s32(xq, wq, acc, stream=None) -> None:

@@ -1,0 +1,394 @@
+// int8 attention for the DiT blocks (h3-rs README, "What makes it fast": an
+// int8 Q.K^T / 16-bit P.V flash kernel). Per head (head dim 128, columns
+// h*128 .. h*128+127 of the [S, ld] q, k, v and out matrices):
+//   Q and K rows are quantized per token (s = max|x| / 127 in fp32, codes
+//   clamp(rne(x / s)), as the weight rows of the linear layers);
+//   s_ij = acc_ij * qs_i * ks_j / sqrt(128) with acc the exact int32 dot product;
+//   O_i = softmax_j(s_i) V, with P in bf16 and fp32 accumulation.
+//
+// attn_prep_kernel: one block per (64-token tile, head): Q and K codes and
+// scales, and V transposed per head (V^T [H*128, S]) so both products read
+// K-major operands.
+//
+// attn_kernel: one CTA per (head, 128-query block); warp roles:
+//   warp 0   TMA: the Q tile once, then K and V^T tiles of 128 keys through a
+//            two-stage ring;
+//   warp 1   tensor memory (512 columns: two 128-column score buffers and the
+//            128-column output accumulator O); one lane issues S_j = Q K_j^T
+//            (kind::i8, 128 x 128 x 128) into score buffer j % 2, then
+//            O += P_{j-1} V_{j-1} (kind::f16, bf16 in, fp32 accumulation),
+//            so S_j is computed while the softmax works on block j-1;
+//   warps 2-5 softmax, one thread per query row (tensor-memory lane): reads
+//            its score row, scales it into the log2 domain, keeps a running
+//            maximum m and sum l, writes P = 2^(s - m) as bf16 into a 128-byte
+//            swizzled shared-memory tile, and at the end writes O / l as bf16.
+//            The maximum used for the exponent is raised only when a row's
+//            maximum grows by more than 2^8 (P stays below 256); O is then
+//            rescaled in tensor memory after the previous P.V has completed.
+// Every wait is bounded (the kernel records a timeout and drains).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "gemm_sm100.cuh"
+#include "ptx_sm100.cuh"
+
+namespace h3q {
+
+constexpr int kAttD = 128;                 // head dimension
+constexpr int kAttBlk = 128;               // queries per CTA, keys per block
+constexpr int kAttQBytes = 128 * 128;      // int8 Q tile
+constexpr int kAttKBytes = 128 * 128;      // int8 K tile
+constexpr int kAttVBytes = 2 * 128 * 128;  // bf16 V^T tile (128 d rows x 128 keys), two 64-key boxes
+constexpr int kAttPBytes = 2 * 128 * 128;  // bf16 P tile (128 rows x 128 keys), two 64-key halves
+constexpr int kAttStages = 2;
+constexpr int kAttThreads = 192;
+constexpr size_t kAttSmem = size_t(kAttQBytes) + kAttStages * (kAttKBytes + kAttVBytes) + 2 * kAttPBytes + 1024 + 256;
+
+struct AttParams {
+  int S, H;
+  const float* qs;       // [H, S]
+  const float* ks;       // [H, S]
+  __nv_bfloat16* out;    // [S, ld_out], head h at columns h*128
+  int64_t ld_out;
+  float c;               // log2(e) / sqrt(128)
+  uint64_t wait_limit_ns;
+};
+
+// Each lane of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32, one CTA.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// kind::f16 with bf16 A and B, fp32 accumulator, K-major operands.
+__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N) {
+  return (1u << 4)             // D format: f32
+         | (1u << 7)           // A format: bf16
+         | (1u << 10)          // B format: bf16
+         | ((N >> 3) << 17)
+         | ((M >> 4) << 24);
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------- prep
+// Block (tile of 64 tokens, head h), 256 threads. Q/K rows: one warp per token
+// (4 elements per lane); V: staged in shared memory and written transposed.
+__global__ void __launch_bounds__(256) attn_prep_kernel(const __nv_bfloat16* __restrict__ q,
+                                                        const __nv_bfloat16* __restrict__ k,
+                                                        const __nv_bfloat16* __restrict__ v, int S, int64_t ld,
+                                                        int8_t* __restrict__ qq, float* __restrict__ qs,
+                                                        int8_t* __restrict__ kq, float* __restrict__ ks,
+                                                        __nv_bfloat16* __restrict__ vt) {
+  __shared__ uint16_t tile[64][kAttD + 2];  // +2 halves: column reads spread over banks
+  const int h = blockIdx.y;
+  const int t0 = blockIdx.x * 64;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t = warp; t < 64; t += 8) {
+    const int i = t0 + t;
+    if (i >= S) break;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const __nv_bfloat16* src = (which == 0 ? q : k) + int64_t(i) * ld + h * kAttD + 4 * lane;
+      const uint2 w = *reinterpret_cast<const uint2*>(src);
+      const float x[4] = {__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u),
+                          __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u)};
+      float a = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+      const float s = __fdiv_rn(a, 127.0f);
+      uint32_t packed = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float r = 0.0f;
+        if (s != 0.0f) r = fminf(fmaxf(rintf(__fdiv_rn(x[e], s)), -127.0f), 127.0f);
+        packed |= (static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu) << (8 * e);
+      }
+      const int64_t row = int64_t(h) * S + i;
+      *reinterpret_cast<uint32_t*>((which == 0 ? qq : kq) + row * kAttD + 4 * lane) = packed;
+      if (lane == 0) (which == 0 ? qs : ks)[row] = s;
+    }
+  }
+  // V tile [64 tokens][128 d] -> V^T rows h*128 + d, columns t0 .. t0+63
+  for (int e = threadIdx.x; e < 64 * (kAttD / 2); e += 256) {
+    const int t = e / (kAttD / 2), d2 = e % (kAttD / 2);
+    const int i = t0 + t;
+    uint32_t w = 0;
+    if (i < S) w = *reinterpret_cast<const uint32_t*>(v + int64_t(i) * ld + h * kAttD + 2 * d2);
+    tile[t][2 * d2] = static_cast<uint16_t>(w & 0xFFFFu);
+    tile[t][2 * d2 + 1] = static_cast<uint16_t>(w >> 16);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kAttD * 32; e += 256) {
+    const int d = e / 32, t2 = e % 32;  // tokens 2 t2, 2 t2 + 1
+    const int i = t0 + 2 * t2;
+    if (i >= S) continue;
+    const uint32_t w = uint32_t(tile[2 * t2][d]) | (uint32_t(tile[2 * t2 + 1][d]) << 16);
+    *reinterpret_cast<uint32_t*>(vt + (int64_t(h) * kAttD + d) * S + i) = w;
+  }
+}
+
+// ---------------------------------------------------------------- attention
+__global__ void __launch_bounds__(kAttThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + kAttQBytes;                   // [stage][128 keys x 128 B]
+  uint8_t* sV = sK + kAttStages * kAttKBytes;      // [stage][2 boxes: 128 d rows x 64 keys (128 B)]
+  uint8_t* sP = sV + kAttStages * kAttVBytes;      // [buffer][2 halves: 128 rows x 64 keys (128 B)]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kAttPBytes);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_empty = bars + 7;   // [2]
+  uint64_t* p_full = bars + 9;    // [2]
+  uint64_t* pv_done = bars + 11;  // [2]
+  uint64_t* drain = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, qb = blockIdx.x;
+  const int S = p.S;
+  const int nb = (S + kAttBlk - 1) / kAttBlk;
+  const uint64_t limit = p.wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&kv_full[b], 1);
+      mbar_init(&kv_empty[b], 1);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], 4);
+      mbar_init(&p_full[b], 4);
+      mbar_init(&pv_done[b], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      const uint64_t pol_q = policy_evict_first();
+      const uint64_t pol_kv = policy_evict_last();  // every query block of the head re-reads K and V
+      mbar_arrive_expect_tx(q_full, kAttQBytes);
+      tma_load_2d(sQ, &tmQ, q_full, 0, h * S + qb * kAttBlk, pol_q);
+      for (int j = 0; j < nb; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait_bounded(&kv_empty[st], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), limit, abort_flag)) break;
+        mbar_arrive_expect_tx(&kv_full[st], kAttKBytes + kAttVBytes);
+        tma_load_2d(sK + st * kAttKBytes, &tmK, &kv_full[st], 0, h * S + j * kAttBlk, pol_kv);
+        tma_load_2d(sV + st * kAttVBytes, &tmV, &kv_full[st], j * kAttBlk, h * kAttD, pol_kv);
+        tma_load_2d(sV + st * kAttVBytes + kAttVBytes / 2, &tmV, &kv_full[st], j * kAttBlk + 64, h * kAttD, pol_kv);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc_s = idesc_i8(kAttBlk, kAttBlk);
+      constexpr uint32_t idesc_o = idesc_bf16(kAttBlk, kAttD);
+      bool ok = mbar_wait_bounded(q_full, 0, limit, abort_flag);
+      const uint64_t qd = smem_desc_sw128(smem_u32(sQ));
+      for (int j = 0; ok && j <= nb; ++j) {
+        if (j < nb) {  // S_j = Q K_j^T into score buffer j % 2
+          const int st = j & 1;
+          if (!mbar_wait_bounded(&kv_full[st], static_cast<uint32_t>((j >> 1) & 1), limit, abort_flag) ||
+              !mbar_wait_bounded(&s_empty[st], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), limit, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t kd = smem_desc_sw128(smem_u32(sK + st * kAttKBytes));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) mma_i8(tmem + st * kAttBlk, qd + 2u * k, kd + 2u * k, idesc_s, k > 0 ? 1u : 0u);
+          mma_commit(&s_full[st]);
+        }
+        if (j >= 1) {  // O += P_{j-1} V_{j-1}
+          const int t = j - 1, bt = t & 1;
+          if (!mbar_wait_bounded(&p_full[bt], static_cast<uint32_t>((t >> 1) & 1), limit, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {  // 16 keys = 32 bytes per K step; halves of 64 keys
+            const int half = k >> 2;
+            const uint64_t pd = smem_desc_sw128(smem_u32(sP + bt * kAttPBytes + half * (kAttPBytes / 2)));
+            const uint64_t vd = smem_desc_sw128(smem_u32(sV + bt * kAttVBytes + half * (kAttVBytes / 2)));
+            mma_bf16(tmem + 2 * kAttBlk, pd + 2u * (k & 3), vd + 2u * (k & 3), idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&pv_done[bt]);
+          mma_commit(&kv_empty[bt]);
+        }
+      }
+      mma_commit(drain);
+      mbar_wait_bounded(drain, 0, limit, nullptr);
+    }
+  } else {
+    // -------------------------------------------------------------- softmax (warps 2..5)
+    const int quarter = warp & 3;                     // TMEM lanes 32*quarter .. +31
+    const int r = quarter * 32 + lane;                // query row within the block
+    const int i = qb * kAttBlk + r;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const float cq = __fmul_rn(i < S ? __ldg(p.qs + int64_t(h) * S + i) : 0.0f, p.c);
+    const float* ksh = p.ks + int64_t(h) * S;
+    float m_used = -INFINITY, l = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nb; ++j) {
+      const int b = j & 1;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&s_full[b], static_cast<uint32_t>((j >> 1) & 1), limit,
+                                                       abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tmem + lane_base + b * kAttBlk + 32 * c4, sr[c4]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[b]);
+      // scores in log2 units: ((float)acc * qs_i * log2(e) / sqrt(128)) * ks_j; -inf past the last key
+      const int key0 = j * kAttBlk;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const int key = key0 + 32 * c4 + 4 * e4;
+          float4 kv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          if (key < S) kv = __ldg(reinterpret_cast<const float4*>(ksh + key));  // S % 8 == 0: whole float4 valid
+          const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * e4 + e;
+            const float s = key < S ? __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(sr[c4][c])), cq), kk[e])
+                                    : -INFINITY;
+            sr[c4][c] = __float_as_uint(s);
+            mx = fmaxf(mx, s);
+          }
+        }
+      }
+      const bool need = mx > m_used + 8.0f;
+      if (__ballot_sync(0xFFFFFFFFu, need) != 0u && j > 0) {
+        // O holds P.V of blocks < j with the old maximum: rescale after P_{j-1} V_{j-1} has landed
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&pv_done[(j - 1) & 1], static_cast<uint32_t>(((j - 1) >> 1) & 1),
+                                                         limit, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const float f = need ? ex2_approx(m_used - mx) : 1.0f;
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + 2 * kAttBlk + 32 * c4, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), f));
+          tmem_st32(tmem + lane_base + 2 * kAttBlk + 32 * c4, o);
+        }
+        tmem_st_wait();
+        l = __fmul_rn(l, f);
+      }
+      if (need) m_used = mx;
+      if (j >= 2) {  // P buffer b was last read by P_{j-2} V_{j-2}
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&pv_done[b], static_cast<uint32_t>(((j - 2) >> 1) & 1), limit,
+                                                         abort_flag));
+        if (!ok) break;
+      }
+      // P = 2^(s - m) as bf16 into row r of the swizzled tile (16-byte chunk c at
+      // position c ^ (r % 8) of the 128-byte row); l sums the rounded values
+      uint8_t* prow = sP + b * kAttPBytes + r * 128;
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c0 = 8 * ch + 2 * e;
+          const float p0 = ex2_approx(__uint_as_float(sr[c0 >> 5][c0 & 31]) - m_used);
+          const float p1 = ex2_approx(__uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]) - m_used);
+          w[e] = pack_bf16x2(p0, p1);
+          l = __fadd_rn(l, __fadd_rn(bf16_bits_to_f32(w[e] & 0xFFFFu), bf16_bits_to_f32(w[e] >> 16)));
+        }
+        const int half = ch >> 3, c8 = ch & 7;
+        *reinterpret_cast<uint4*>(prow + half * (kAttPBytes / 2) + 16 * (c8 ^ (r & 7))) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();  // the tensor core reads P through the async proxy
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[b]);
+    }
+    if (ok) {
+      const int t = nb - 1;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&pv_done[t & 1], static_cast<uint32_t>((t >> 1) & 1), limit,
+                                                       abort_flag));
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = __fdiv_rn(1.0f, l);
+      __nv_bfloat16* orow = p.out + int64_t(i) * p.ld_out + h * kAttD;
+#pragma unroll 1
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + 2 * kAttBlk + 32 * c4, o);
+        tmem_ld_wait();
+        if (i < S) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack_bf16x2(__fmul_rn(__uint_as_float(o[8 * g + 2 * e]), inv_l),
+                                 __fmul_rn(__uint_as_float(o[8 * g + 2 * e + 1]), inv_l));
+            *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace h3q

@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <mutex>
 
@@ -14,6 +15,7 @@
 #include "gemm_sm100.cuh"
 #include "lora.cuh"
 #include "nvfp4.cuh"
+#include "attention.cuh"
 #include "rotquant.cuh"
 
 namespace {
@@ -166,6 +168,20 @@ h3q_status launch_gemm_fp4(const uint8_t* a, const uint8_t* a_sf, const float* a
   const int pairs = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
   h3q::gemm_fp4_kernel<EPI><<<2 * pairs, h3q::kGemmThreads, h3q::kF4Smem, stream>>>(ta, tb, tsa, tsb, p);
   return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+}
+
+// [rows, cols] bf16 row-major, boxes of 64 columns (128 bytes) x 128 rows,
+// 128-byte swizzle; reads past the edges return zeros.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool valid_k(int64_t K) { return K >= 256 && K % 256 == 0; }
@@ -348,6 +364,93 @@ h3q_status h3q_gemm_nvfp4_f32(const uint8_t* xc, const uint8_t* xsf, int64_t M, 
   if (st != H3Q_OK || M == 0) return st;
   if (!acc || !aligned16(acc)) return H3Q_ERR_INVALID_ARG;
   return launch_gemm_fp4<h3q::kEpiS32>(xc, xsf, nullptr, M, K, wc, wsf, nullptr, N, N, nullptr, acc, stream);
+}
+
+struct AttLayout {
+  size_t qq, kq, qs, ks, vt, total;
+};
+
+AttLayout att_layout(int64_t S, int64_t H) {
+  AttLayout l{};
+  const size_t codes = size_t(H) * S * 128, scales = size_t(H) * S * 4, vt = size_t(H) * 128 * S * 2;
+  l.qq = 0;
+  l.kq = align256(l.qq + codes);
+  l.qs = align256(l.kq + codes);
+  l.ks = align256(l.qs + scales);
+  l.vt = align256(l.ks + scales);
+  l.total = align256(l.vt + vt);
+  return l;
+}
+
+static h3q_status check_att_args(const void* q, const void* k, const void* v, int64_t S, int64_t H, int64_t ld) {
+  if (S < 0 || H < 1 || S % 8 != 0 || ld < H * 128 || ld % 8 != 0) return H3Q_ERR_INVALID_ARG;
+  if (H * S > INT32_MAX / 2 || S > INT32_MAX - 256) return H3Q_ERR_UNSUPPORTED;
+  if (S == 0) return H3Q_OK;
+  if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return H3Q_ERR_INVALID_ARG;
+  return H3Q_OK;
+}
+
+size_t h3q_attention_workspace_size(int64_t S, int64_t H) {
+  if (S < 0 || H < 1) return 0;
+  return att_layout(S, H).total;
+}
+
+h3q_status h3q_attention_prep(const void* q, const void* k, const void* v, int64_t S, int64_t H, int64_t ld,
+                              int8_t* qq, float* qs, int8_t* kq, float* ks, void* vt, cudaStream_t stream) {
+  const h3q_status st = check_att_args(q, k, v, S, H, ld);
+  if (st != H3Q_OK || S == 0) return st;
+  if (!qq || !qs || !kq || !ks || !vt || !aligned16(qq) || !aligned16(qs) || !aligned16(kq) || !aligned16(ks) ||
+      !aligned16(vt))
+    return H3Q_ERR_INVALID_ARG;
+  const dim3 grid(static_cast<unsigned>((S + 63) / 64), static_cast<unsigned>(H));
+  h3q::attn_prep_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q),
+                                                  static_cast<const __nv_bfloat16*>(k),
+                                                  static_cast<const __nv_bfloat16*>(v), static_cast<int>(S), ld, qq,
+                                                  qs, kq, ks, static_cast<__nv_bfloat16*>(vt));
+  return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+}
+
+h3q_status h3q_attention_int8(const void* q, const void* k, const void* v, int64_t S, int64_t H, int64_t ld,
+                              void* out, int64_t ld_out, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+  h3q_status st = check_att_args(q, k, v, S, H, ld);
+  if (st != H3Q_OK || S == 0) return st;
+  if (!out || !aligned16(out) || ld_out < H * 128 || ld_out % 8 != 0 || !workspace ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return H3Q_ERR_INVALID_ARG;
+  const AttLayout lay = att_layout(S, H);
+  if (workspace_bytes < lay.total) return H3Q_ERR_INVALID_ARG;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* qq = reinterpret_cast<int8_t*>(ws + lay.qq);
+  int8_t* kq = reinterpret_cast<int8_t*>(ws + lay.kq);
+  float* qs = reinterpret_cast<float*>(ws + lay.qs);
+  float* ks = reinterpret_cast<float*>(ws + lay.ks);
+  void* vt = ws + lay.vt;
+  st = h3q_attention_prep(q, k, v, S, H, ld, qq, qs, kq, ks, vt, stream);
+  if (st != H3Q_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_i8(&tq, qq, H * S, 128) || !make_tmap_i8(&tk, kq, H * S, 128) ||
+      !make_tmap_bf16(&tv, vt, H * 128, S))
+    return H3Q_ERR_CUDA;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(h3q::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(h3q::kAttSmem));
+  });
+  if (attr_err != cudaSuccess) return H3Q_ERR_CUDA;
+  h3q::AttParams p{};
+  p.S = static_cast<int>(S);
+  p.H = static_cast<int>(H);
+  p.qs = qs;
+  p.ks = ks;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.ld_out = ld_out;
+  p.c = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const dim3 grid(static_cast<unsigned>((S + 127) / 128), static_cast<unsigned>(H));
+  h3q::attn_kernel<<<grid, h3q::kAttThreads, h3q::kAttSmem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
 }
 
 h3q_status h3q_gemm_s32(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N, int64_t K, int32_t* acc,
