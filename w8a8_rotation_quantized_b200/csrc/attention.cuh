@@ -18,10 +18,12 @@
 //            (kind::i8, 128 x 128 x 128) into score buffer j % 2, then
 //            O += P_{j-1} V_{j-1} (kind::f16, bf16 in, fp32 accumulation),
 //            so S_j is computed while the softmax works on block j-1;
-//   warps 2-5 softmax, one thread per query row (tensor-memory lane): reads
-//            its score row, scales it into the log2 domain, keeps a running
-//            maximum m and sum l, writes P = 2^(s - m) as bf16 into a 128-byte
-//            swizzled shared-memory tile, and at the end writes O / l as bf16.
+//   warps 2-9 softmax, two threads per query row (tensor-memory lane), each
+//            with 64 keys of the block: reads its half score row, scales it
+//            into the log2 domain (key scales staged in shared memory with the
+//            K tile), exchanges the half-row maxima, keeps a running maximum m
+//            and sum l, writes P = 2^(s - m) as bf16 into its 128-byte swizzled
+//            half-tile, and at the end writes its half of O / l as bf16.
 //            The maximum used for the exponent is raised only when a row's
 //            maximum grows by more than 2^8 (P stays below 256); O is then
 //            rescaled in tensor memory after the previous P.V has completed.
@@ -44,8 +46,11 @@ constexpr int kAttKBytes = 128 * 128;      // int8 K tile
 constexpr int kAttVBytes = 2 * 128 * 128;  // bf16 V^T tile (128 d rows x 128 keys), two 64-key boxes
 constexpr int kAttPBytes = 2 * 128 * 128;  // bf16 P tile (128 rows x 128 keys), two 64-key halves
 constexpr int kAttStages = 2;
-constexpr int kAttThreads = 192;
-constexpr size_t kAttSmem = size_t(kAttQBytes) + kAttStages * (kAttKBytes + kAttVBytes) + 2 * kAttPBytes + 1024 + 256;
+constexpr int kAttThreads = 320;  // producer, MMA, 8 softmax warps (two threads per query row)
+constexpr int kAttKsBytes = 128 * 4;  // the key block's scales
+constexpr size_t kAttSmem = size_t(kAttQBytes) + kAttStages * (kAttKBytes + kAttVBytes + kAttKsBytes) +
+                            2 * kAttPBytes + 2 * 2 * 128 * 4 /*row max exchange*/ + 2 * 128 * 4 /*row sums*/ +
+                            1024 + 256;
 
 struct AttParams {
   int S, H;
@@ -164,7 +169,10 @@ __global__ void __launch_bounds__(kAttThreads, 1)
   uint8_t* sK = sQ + kAttQBytes;                   // [stage][128 keys x 128 B]
   uint8_t* sV = sK + kAttStages * kAttKBytes;      // [stage][2 boxes: 128 d rows x 64 keys (128 B)]
   uint8_t* sP = sV + kAttStages * kAttVBytes;      // [buffer][2 halves: 128 rows x 64 keys (128 B)]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kAttPBytes);
+  float* sKs = reinterpret_cast<float*>(sP + 2 * kAttPBytes);  // [stage][128] key scales
+  float* xmax = sKs + kAttStages * 128;            // [block parity][half][128 rows]: half-row maxima
+  float* xsum = xmax + 2 * 2 * 128;                // [half][128 rows]: half-row sums at the end
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xsum + 2 * 128);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;   // [2]
   uint64_t* kv_empty = bars + 3;  // [2]
@@ -173,7 +181,9 @@ __global__ void __launch_bounds__(kAttThreads, 1)
   uint64_t* p_full = bars + 9;    // [2]
   uint64_t* pv_done = bars + 11;  // [2]
   uint64_t* drain = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* xchg = bars + 14;     // [2]: the 256 softmax threads exchanged their half-row maxima
+  uint64_t* xsum_bar = bars + 16; // the 256 softmax threads stored their half-row sums
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,11 +198,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       mbar_init(&kv_full[b], 1);
       mbar_init(&kv_empty[b], 1);
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 4);
-      mbar_init(&p_full[b], 4);
+      mbar_init(&s_empty[b], 8);
+      mbar_init(&p_full[b], 8);
       mbar_init(&pv_done[b], 1);
+      mbar_init(&xchg[b], 256);
     }
     mbar_init(drain, 1);
+    mbar_init(xsum_bar, 256);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -215,7 +227,9 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       for (int j = 0; j < nb; ++j) {
         const int st = j & 1;
         if (!mbar_wait_bounded(&kv_empty[st], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), limit, abort_flag)) break;
-        mbar_arrive_expect_tx(&kv_full[st], kAttKBytes + kAttVBytes);
+        const uint32_t ks_bytes = static_cast<uint32_t>(min(kAttBlk, S - j * kAttBlk) * 4);  // S % 8 == 0
+        mbar_arrive_expect_tx(&kv_full[st], kAttKBytes + kAttVBytes + ks_bytes);
+        bulk_load(sKs + st * 128, p.ks + int64_t(h) * S + j * kAttBlk, ks_bytes, &kv_full[st], pol_kv);
         tma_load_2d(sK + st * kAttKBytes, &tmK, &kv_full[st], 0, h * S + j * kAttBlk, pol_kv);
         tma_load_2d(sV + st * kAttVBytes, &tmV, &kv_full[st], j * kAttBlk, h * kAttD, pol_kv);
         tma_load_2d(sV + st * kAttVBytes + kAttVBytes / 2, &tmV, &kv_full[st], j * kAttBlk + 64, h * kAttD, pol_kv);
@@ -264,80 +278,88 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       mbar_wait_bounded(drain, 0, limit, nullptr);
     }
   } else {
-    // -------------------------------------------------------------- softmax (warps 2..5)
+    // -------------------------------------------------------------- softmax (warps 2..9)
+    // Two threads per query row (TMEM lane): warps 2-5 take keys [0, 64) of each
+    // block and columns [0, 64) of O, warps 6-9 keys [64, 128) and columns [64, 128).
+    // The two halves exchange their row maxima through shared memory and a
+    // 256-arrival mbarrier per block, so both take the same rescale decisions.
     const int quarter = warp & 3;                     // TMEM lanes 32*quarter .. +31
+    const int half = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;                // query row within the block
     const int i = qb * kAttBlk + r;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float cq = __fmul_rn(i < S ? __ldg(p.qs + int64_t(h) * S + i) : 0.0f, p.c);
-    const float* ksh = p.ks + int64_t(h) * S;
     float m_used = -INFINITY, l = 0.0f;
     bool ok = true;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xFFFFFFFFu, mbar_wait_bounded(bar, parity, limit, abort_flag));
+    };
     for (int j = 0; j < nb; ++j) {
-      const int b = j & 1;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&s_full[b], static_cast<uint32_t>((j >> 1) & 1), limit,
-                                                       abort_flag));
-      if (!ok) break;
+      const int b = j & 1, st = j & 1;
+      if (!(ok = wait_all(&s_full[b], static_cast<uint32_t>((j >> 1) & 1)))) break;
       tc_fence_after();
-      uint32_t sr[4][32];
+      uint32_t sr[2][32];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tmem + lane_base + b * kAttBlk + 32 * c4, sr[c4]);
+      for (int c2 = 0; c2 < 2; ++c2) tmem_ld32(tmem + lane_base + b * kAttBlk + 64 * half + 32 * c2, sr[c2]);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[b]);
-      // scores in log2 units: ((float)acc * qs_i * log2(e) / sqrt(128)) * ks_j; -inf past the last key
-      const int key0 = j * kAttBlk;
+      // scores in log2 units: (float)acc * (qs_i * log2(e) / sqrt(128) * ks_j); -inf past the last key
+      const int key0 = j * kAttBlk + 64 * half;
+      const float* ksb = sKs + st * 128 + 64 * half;
       float mx = -INFINITY;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c2 = 0; c2 < 2; ++c2) {
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
-          const int key = key0 + 32 * c4 + 4 * e4;
-          float4 kv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          if (key < S) kv = __ldg(reinterpret_cast<const float4*>(ksh + key));  // S % 8 == 0: whole float4 valid
+          const float4 kv = *reinterpret_cast<const float4*>(ksb + 32 * c2 + 4 * e4);
           const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = 4 * e4 + e;
-            const float s = key < S ? __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(sr[c4][c])), cq), kk[e])
-                                    : -INFINITY;
-            sr[c4][c] = __float_as_uint(s);
-            mx = fmaxf(mx, s);
+            // |acc| <= 127^2 * 128 < 2^22: the bits of acc + 1.5 * 2^23 read as a
+            // float, minus 1.5 * 2^23, give (float)acc exactly without the conversion unit
+            const float af = __fsub_rn(__uint_as_float(sr[c2][c] + 0x4B400000u), 12582912.0f);
+            const float sc = key0 + 32 * c2 + c < S ? __fmul_rn(af, __fmul_rn(cq, kk[e])) : -INFINITY;
+            sr[c2][c] = __float_as_uint(sc);
+            mx = fmaxf(mx, sc);
           }
         }
       }
+      float* xm = xmax + b * 256;
+      xm[half * 128 + r] = mx;
+      mbar_arrive(&xchg[b]);
+      if (!(ok = wait_all(&xchg[b], static_cast<uint32_t>((j >> 1) & 1)))) break;
+      mx = fmaxf(mx, xm[(1 - half) * 128 + r]);
       const bool need = mx > m_used + 8.0f;
       if (__ballot_sync(0xFFFFFFFFu, need) != 0u && j > 0) {
         // O holds P.V of blocks < j with the old maximum: rescale after P_{j-1} V_{j-1} has landed
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&pv_done[(j - 1) & 1], static_cast<uint32_t>(((j - 1) >> 1) & 1),
-                                                         limit, abort_flag));
-        if (!ok) break;
+        if (!(ok = wait_all(&pv_done[(j - 1) & 1], static_cast<uint32_t>(((j - 1) >> 1) & 1)))) break;
         tc_fence_after();
         const float f = need ? ex2_approx(m_used - mx) : 1.0f;
 #pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
+        for (int c2 = 0; c2 < 2; ++c2) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_base + 2 * kAttBlk + 32 * c4, o);
+          const uint32_t oaddr = tmem + lane_base + 2 * kAttBlk + 64 * half + 32 * c2;
+          tmem_ld32(oaddr, o);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), f));
-          tmem_st32(tmem + lane_base + 2 * kAttBlk + 32 * c4, o);
+          tmem_st32(oaddr, o);
         }
         tmem_st_wait();
         l = __fmul_rn(l, f);
       }
       if (need) m_used = mx;
       if (j >= 2) {  // P buffer b was last read by P_{j-2} V_{j-2}
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&pv_done[b], static_cast<uint32_t>(((j - 2) >> 1) & 1), limit,
-                                                         abort_flag));
-        if (!ok) break;
+        if (!(ok = wait_all(&pv_done[b], static_cast<uint32_t>(((j - 2) >> 1) & 1)))) break;
       }
-      // P = 2^(s - m) as bf16 into row r of the swizzled tile (16-byte chunk c at
+      // P = 2^(s - m) as bf16 into row r of the half-tile (16-byte chunk c at
       // position c ^ (r % 8) of the 128-byte row); l sums the rounded values
-      uint8_t* prow = sP + b * kAttPBytes + r * 128;
+      uint8_t* prow = sP + b * kAttPBytes + half * (kAttPBytes / 2) + r * 128;
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
+      for (int ch = 0; ch < 8; ++ch) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -347,9 +369,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
           w[e] = pack_bf16x2(p0, p1);
           l = __fadd_rn(l, __fadd_rn(bf16_bits_to_f32(w[e] & 0xFFFFu), bf16_bits_to_f32(w[e] >> 16)));
         }
-        const int half = ch >> 3, c8 = ch & 7;
-        *reinterpret_cast<uint4*>(prow + half * (kAttPBytes / 2) + 16 * (c8 ^ (r & 7))) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(prow + 16 * (ch ^ (r & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();  // the tensor core reads P through the async proxy
       tc_fence_before();
@@ -358,17 +378,21 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     }
     if (ok) {
       const int t = nb - 1;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&pv_done[t & 1], static_cast<uint32_t>((t >> 1) & 1), limit,
-                                                       abort_flag));
+      ok = wait_all(&pv_done[t & 1], static_cast<uint32_t>((t >> 1) & 1));
+    }
+    if (ok) {
+      xsum[half * 128 + r] = l;
+      mbar_arrive(xsum_bar);
+      ok = wait_all(xsum_bar, 0);
     }
     if (ok) {
       tc_fence_after();
-      const float inv_l = __fdiv_rn(1.0f, l);
-      __nv_bfloat16* orow = p.out + int64_t(i) * p.ld_out + h * kAttD;
+      const float inv_l = __fdiv_rn(1.0f, __fadd_rn(xsum[r], xsum[128 + r]));
+      __nv_bfloat16* orow = p.out + int64_t(i) * p.ld_out + h * kAttD + 64 * half;
 #pragma unroll 1
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_base + 2 * kAttBlk + 32 * c4, o);
+        tmem_ld32(tmem + lane_base + 2 * kAttBlk + 64 * half + 32 * c2, o);
         tmem_ld_wait();
         if (i < S) {
 #pragma unroll
@@ -378,7 +402,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             for (int e = 0; e < 4; ++e)
               w[e] = pack_bf16x2(__fmul_rn(__uint_as_float(o[8 * g + 2 * e]), inv_l),
                                  __fmul_rn(__uint_as_float(o[8 * g + 2 * e + 1]), inv_l));
-            *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(orow + 32 * c2 + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
