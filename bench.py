@@ -27,6 +27,11 @@ Workload nvfp4: the hybrid checkpoints' four linear operations of one block at
 INT8 ConvRot, each with the quantization of its input), next to the same four
 operations all in INT8 ConvRot; value in TOPS of the four GEMMs.
 
+Workload attention: the DiT attention call at 16384 tokens, 42 heads of 128
+(int8 Q.K^T, bf16 P.V), from a QKV projection output; value in TFLOP/s of the
+two products (4 S^2 D H); the library's bf16 scaled-dot-product attention on
+the same tensors is timed beside it as context.
+
 Multi-GPU (torchrun): every rank runs its own batch with replicated weights
 (the rows are independent; there is no data-path collective). Times are the
 max over ranks; the value is the work of all ranks over that time.
@@ -57,7 +62,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="h3q", choices=["h3q", "reference"])
-    ap.add_argument("--workload", default="ffn", choices=["ffn", "qkv", "out", "tiny", "sweep", "lora", "nvfp4"])
+    ap.add_argument("--workload", default="ffn", choices=["ffn", "qkv", "out", "tiny", "sweep", "lora", "nvfp4", "attention"])
     ap.add_argument("--M", type=int, default=None, help="tokens per GPU (default: the workload's)")
     ap.add_argument("--F", type=int, default=None, help="FFN width (default 14336)")
     ap.add_argument("--kernel-reps", type=int, default=10)
@@ -248,6 +253,23 @@ def run_reference(args):
     import oracle
     import synth
 
+    if args.workload == "attention":
+        per_step = 60.0 / max(1, args.steps + args.warmup)
+        S = args.M or 16384
+        for _ in range(args.warmup):
+            oracle_attention_rate(S, 42, per_step)
+        vals = [oracle_attention_rate(S, 42, per_step) for _ in range(args.steps)]
+        secs = sum(v["seconds"] for v in vals)
+        value = sum(v["value"] * v["seconds"] for v in vals) / secs
+        line = {"impl": "reference", "metric": "int8 attention TFLOP/s", "value": value, "unit": "TFLOP/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8+bf16",
+                "data": "synthetic", "config": {"workload": f"DiT attention S={S}, 42 heads, sampled query rows"},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                                 "sample": vals[-1]["sample"]},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
     if args.workload == "nvfp4":
         per_step = 60.0 / max(1, args.steps + args.warmup)
         for _ in range(args.warmup):
@@ -780,6 +802,139 @@ def oracle_nvfp4_rate(target_s):
             "sample": f"{rows} token rows of the QKV projection in NVFP4 (full weight), {dt:.1f} s"}
 
 
+def run_attention(args):
+    """int8 attention of one DiT block (S tokens, 42 heads of 128) from a QKV output."""
+    import torch
+    import torch.distributed as dist
+
+    import w8a8_rotation_quantized_b200 as h3q
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    S = args.M or 16384
+    H, D = 42, 128
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    qkv = torch.randn((S, 3 * H * D), device=dev, dtype=torch.float32, generator=gen).to(torch.bfloat16)
+    q, k, v = qkv[:, :H * D], qkv[:, H * D:2 * H * D], qkv[:, 2 * H * D:]
+    out = torch.empty((S, H * D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(h3q.h3q_attention_workspace_size(S, H), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        h3q.h3q_attention_int8(q, k, v, H, out, ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, n):
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for i in range(n):
+            flush.fill_(i & 0xFF)
+            st[i].record(stream)
+            fn()
+            en[i].record(stream)
+        barrier()
+        return sum(a.elapsed_time(b) for a, b in zip(st, en))
+
+    steps = max(1, min(args.steps, 20))
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.5)
+    t_host0 = time.time()
+    total_ms = max_over_ranks(timed(step, steps), dev)
+    clk = clocks.stop(t_host0, time.time())
+    st = h3q.h3q_get_device_status()
+    if st != h3q.H3Q_OK:
+        raise RuntimeError(f"device status after the timed region: {h3q.h3q_status_string(st)}")
+    qh, kh, vh = (t.reshape(S, H, D).transpose(0, 1)[None].contiguous() for t in (q, k, v))
+    sdpa_ms, sdpa_backend = None, None
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    for backend in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION):
+        try:
+            with sdpa_kernel([backend]):
+                torch.nn.functional.scaled_dot_product_attention(qh, kh, vh)
+                torch.cuda.synchronize()
+                sdpa_ms = max_over_ranks(
+                    timed(lambda: torch.nn.functional.scaled_dot_product_attention(qh, kh, vh), 3), dev) / 3
+            sdpa_backend = str(backend).split(".")[-1]
+            break
+        except RuntimeError:
+            continue
+    if rank == 0:
+        ms = total_ms / steps
+        flops = 4.0 * S * S * D * H
+        peaks, peak_src = measured_peaks()
+        p8, p16 = 2.0 * peaks["bf16_tflops"], peaks["bf16_tflops"]
+        mixed = 2.0 / (1.0 / p8 + 1.0 / p16)  # half the work int8, half bf16
+        achieved = flops / (ms * 1e-3) / 1e12
+        line = {
+            "metric": "int8 attention TFLOP/s", "value": achieved * world, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "i8+bf16", "data": "synthetic",
+            "config": {"workload": f"DiT attention, S={S} tokens, {H} heads x {D} (int8 Q.K^T, bf16 P.V), "
+                                   "q/k/v column slices of one [S, 3*5376] bf16 QKV output, N(0,1)",
+                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+                       "parallelism": f"replicas x{world}"},
+            "context_library_bf16_sdpa": {"ms": sdpa_ms, "backend": sdpa_backend,
+                                          "note": "library bf16 attention on the same tensors; context, not a target"},
+            "roofline": {"bound": "tensor", "kernel": "attn_kernel (+ attn_prep_kernel)", "achieved": achieved,
+                         "peak": mixed, "unit": "TFLOP/s", "frac": achieved / mixed, "traffic": None,
+                         "peak_source": f"{peak_src}: half the flops at the int8 rate (2 x bf16 burst) and half at "
+                                        f"the bf16 burst rate {peaks['bf16_tflops']} TFLOP/s"},
+            "gpu_launches": 2 * steps,
+            "clocks": clk,
+            "e2e": None,
+        }
+        if not args.no_cpu_baseline:
+            try:
+                line["cpu_baseline"] = oracle_attention_rate(S, H, args.cpu_seconds)
+            except Exception as exc:
+                line["cpu_baseline"] = {"value": None, "error": repr(exc)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def oracle_attention_rate(S, H, target_s):
+    """The oracle's int8 attention for a bounded sample of query rows of every head
+    (all S keys); flops of the two products per second."""
+    import numpy as np
+
+    import oracle
+    D = 128
+    rng = np.random.default_rng(0)
+    bits = np.ascontiguousarray(
+        (rng.standard_normal((S, 3 * H * D), dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16))
+    q, k, v = bits[:, :H * D], bits[:, H * D:2 * H * D], bits[:, 2 * H * D:]
+    n = 1
+    while True:
+        t0 = time.perf_counter()
+        oracle.attention_int8(q, k, v, H, rows=np.arange(n))
+        dt = time.perf_counter() - t0
+        if dt >= target_s or n >= S:
+            break
+        n = min(S, max(2 * n, int(n * target_s / max(dt, 1e-3) * 1.1)))
+    return {"value": 4.0 * n * S * D * H / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "rows": n, "seconds": dt,
+            "sample": f"{n} query rows x {H} heads against all {S} keys (includes quantizing all Q/K rows), {dt:.1f} s"}
+
+
 def oracle_lora_rate(target_s, steps=None):
     """The oracle's LoRA merge on a bounded sample of the gate/up weight's rows
     (full K and rank); flops of the low-rank product per second."""
@@ -1071,6 +1226,8 @@ def main():
         return run_lora(args)
     if args.workload == "nvfp4":
         return run_nvfp4(args)
+    if args.workload == "attention":
+        return run_attention(args)
     return run_gpu(args)
 
 
