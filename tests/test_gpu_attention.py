@@ -22,11 +22,13 @@ pytestmark = pytest.mark.gpu
 D = 128
 
 
-def _qkv(S, H, seed, dev, growing=False):
+def _qkv(S, H, seed, dev, growing=False, zero_q_rows=()):
     """One [S, 3 H D] bf16 matrix (a QKV projection output); q, k, v column slices."""
     rng = np.random.default_rng(seed)
     x = rng.standard_normal((S, 3 * H * D), dtype=np.float32)
     x[:, :H * D] *= 1.5
+    for i in zero_q_rows:  # a query row of zeros: its scale is 0, all its scores 0, uniform weights
+        x[i, :D] = 0.0
     if growing:  # keys grow along the sequence: the running maximum keeps moving
         x[:, H * D:2 * H * D] *= np.linspace(0.2, 4.0, S, dtype=np.float32)[:, None]
     t = torch.from_numpy(x).to(dev).bfloat16()
@@ -84,6 +86,16 @@ def test_attention_matches_oracle(cuda_device, S, H, seed):
     t, bits = _qkv(S, H, seed, cuda_device)
     out = _run(h3q, t, S, H)
     _check(out, bits, S, H)
+
+
+def test_zero_query_row_with_ragged_last_block(cuda_device):
+    import w8a8_rotation_quantized_b200 as h3q
+    S, H = 200, 1
+    t, bits = _qkv(S, H, 7, cuda_device, zero_q_rows=(5, 150))
+    out = _run(h3q, t, S, H)
+    _check(out, bits, S, H)
+    mean_v = synth.bf16_bits_to_fp32(bits[:, 2 * D:3 * D]).astype(np.float64).mean(axis=0)
+    assert np.abs(out[5].float().cpu().numpy() - mean_v).max() < 2e-2
 
 
 def test_attention_with_moving_maximum(cuda_device):

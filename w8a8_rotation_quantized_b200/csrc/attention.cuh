@@ -20,10 +20,11 @@
 //            so S_j is computed while the softmax works on block j-1;
 //   warps 2-9 softmax, two threads per query row (tensor-memory lane), each
 //            with 64 keys of the block: reads its half score row, scales it
-//            into the log2 domain (key scales staged in shared memory with the
-//            K tile), exchanges the half-row maxima, keeps a running maximum m
-//            and sum l, writes P = 2^(s - m) as bf16 into its 128-byte swizzled
-//            half-tile, and at the end writes its half of O / l as bf16.
+//            with the key scales (staged in shared memory with the K tile),
+//            exchanges the half-row maxima, keeps a running maximum m and sum l
+//            (fp32, of the unrounded weights), writes P = 2^(s - m) as bf16 into
+//            its 128-byte swizzled half-tile, and at the end writes its half of
+//            O / l as bf16.
 //            The maximum used for the exponent is raised only when a row's
 //            maximum grows by more than 2^8 (P stays below 256); O is then
 //            rescaled in tensor memory after the previous P.V has completed.
@@ -94,6 +95,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N) {
          | (1u << 10)          // B format: bf16
          | ((N >> 3) << 17)
          | ((M >> 4) << 24);
+}
+
+// max of three fp32 values (sm_100 three-input max).
+__device__ __forceinline__ float att_max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -289,7 +297,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     const int i = qb * kAttBlk + r;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float cq = __fmul_rn(i < S ? __ldg(p.qs + int64_t(h) * S + i) : 0.0f, p.c);
-    float m_used = -INFINITY, l = 0.0f;
+    float m_used = -INFINITY;
+    float2 l2 = make_float2(0.0f, 0.0f);  // running sum of the weights, two partial sums
     bool ok = true;
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xFFFFFFFFu, mbar_wait_bounded(bar, parity, limit, abort_flag));
@@ -305,8 +314,12 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[b]);
-      // scores in log2 units: (float)acc * (qs_i * log2(e) / sqrt(128) * ks_j); -inf past the last key
+      // Raw scores s' = (float)acc * ks_j (|acc| <= 127^2 * 128 < 2^22, so the bits of
+      // acc + 1.5 * 2^23 read as a float, minus 1.5 * 2^23, are (float)acc without the
+      // conversion unit); the log2-domain score is s' * cq, cq = qs_i log2(e) / sqrt(128) >= 0,
+      // so maxima can be taken on s'. Keys past the end (last block only) are masked.
       const int key0 = j * kAttBlk + 64 * half;
+      const bool partial = key0 + 64 > S;
       const float* ksb = sKs + st * 128 + 64 * half;
       float mx = -INFINITY;
 #pragma unroll
@@ -315,16 +328,15 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         for (int e4 = 0; e4 < 8; ++e4) {
           const float4 kv = *reinterpret_cast<const float4*>(ksb + 32 * c2 + 4 * e4);
           const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+          float sc[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = 4 * e4 + e;
-            // |acc| <= 127^2 * 128 < 2^22: the bits of acc + 1.5 * 2^23 read as a
-            // float, minus 1.5 * 2^23, give (float)acc exactly without the conversion unit
-            const float af = __fsub_rn(__uint_as_float(sr[c2][c] + 0x4B400000u), 12582912.0f);
-            const float sc = key0 + 32 * c2 + c < S ? __fmul_rn(af, __fmul_rn(cq, kk[e])) : -INFINITY;
-            sr[c2][c] = __float_as_uint(sc);
-            mx = fmaxf(mx, sc);
+            sc[e] = __fmul_rn(__fsub_rn(__uint_as_float(sr[c2][c] + 0x4B400000u), 12582912.0f), kk[e]);
+            if (partial && key0 + 32 * c2 + c >= S) sc[e] = -INFINITY;
+            sr[c2][c] = __float_as_uint(sc[e]);
           }
+          mx = att_max3(mx, att_max3(sc[0], sc[1], sc[2]), sc[3]);
         }
       }
       float* xm = xmax + b * 256;
@@ -332,12 +344,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       mbar_arrive(&xchg[b]);
       if (!(ok = wait_all(&xchg[b], static_cast<uint32_t>((j >> 1) & 1)))) break;
       mx = fmaxf(mx, xm[(1 - half) * 128 + r]);
-      const bool need = mx > m_used + 8.0f;
+      // raise the exponent's maximum when the row maximum grew by more than 2^8 (log2 units)
+      const bool need = j == 0 || __fmul_rn(mx - m_used, cq) > 8.0f;
       if (__ballot_sync(0xFFFFFFFFu, need) != 0u && j > 0) {
         // O holds P.V of blocks < j with the old maximum: rescale after P_{j-1} V_{j-1} has landed
         if (!(ok = wait_all(&pv_done[(j - 1) & 1], static_cast<uint32_t>(((j - 1) >> 1) & 1)))) break;
         tc_fence_after();
-        const float f = need ? ex2_approx(m_used - mx) : 1.0f;
+        const float f = need ? ex2_approx(__fmul_rn(m_used - mx, cq)) : 1.0f;
 #pragma unroll 1
         for (int c2 = 0; c2 < 2; ++c2) {
           uint32_t o[32];
@@ -349,14 +362,15 @@ __global__ void __launch_bounds__(kAttThreads, 1)
           tmem_st32(oaddr, o);
         }
         tmem_st_wait();
-        l = __fmul_rn(l, f);
+        l2 = __fmul2_rn(l2, make_float2(f, f));
       }
       if (need) m_used = mx;
       if (j >= 2) {  // P buffer b was last read by P_{j-2} V_{j-2}
         if (!(ok = wait_all(&pv_done[b], static_cast<uint32_t>(((j - 2) >> 1) & 1)))) break;
       }
-      // P = 2^(s - m) as bf16 into row r of the half-tile (16-byte chunk c at
-      // position c ^ (r % 8) of the 128-byte row); l sums the rounded values
+      // P = 2^(s' cq - m cq) as bf16 into row r of the half-tile (16-byte chunk c at
+      // position c ^ (r % 8) of the 128-byte row); l sums the weights in fp32, in pairs
+      const float nm = -__fmul_rn(m_used, cq);
       uint8_t* prow = sP + b * kAttPBytes + half * (kAttPBytes / 2) + r * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
@@ -364,10 +378,14 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int c0 = 8 * ch + 2 * e;
-          const float p0 = ex2_approx(__uint_as_float(sr[c0 >> 5][c0 & 31]) - m_used);
-          const float p1 = ex2_approx(__uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]) - m_used);
+          float p0 = ex2_approx(__fmaf_rn(__uint_as_float(sr[c0 >> 5][c0 & 31]), cq, nm));
+          float p1 = ex2_approx(__fmaf_rn(__uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]), cq, nm));
+          if (partial) {  // masked keys weigh 0 (also when cq = 0, where -inf * cq is not a number)
+            if (key0 + c0 >= S) p0 = 0.0f;
+            if (key0 + c0 + 1 >= S) p1 = 0.0f;
+          }
           w[e] = pack_bf16x2(p0, p1);
-          l = __fadd_rn(l, __fadd_rn(bf16_bits_to_f32(w[e] & 0xFFFFu), bf16_bits_to_f32(w[e] >> 16)));
+          l2 = __fadd2_rn(l2, make_float2(p0, p1));
         }
         *reinterpret_cast<uint4*>(prow + 16 * (ch ^ (r & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
       }
@@ -381,7 +399,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       ok = wait_all(&pv_done[t & 1], static_cast<uint32_t>((t >> 1) & 1));
     }
     if (ok) {
-      xsum[half * 128 + r] = l;
+      xsum[half * 128 + r] = __fadd_rn(l2.x, l2.y);
       mbar_arrive(xsum_bar);
       ok = wait_all(xsum_bar, 0);
     }
