@@ -11,20 +11,22 @@
 // K-major operands.
 //
 // attn_kernel: one CTA per (head, 128-query block); warp roles:
-//   warp 0   TMA: the Q tile once, then K and V^T tiles of 128 keys through a
-//            two-stage ring;
+//   warp 0   TMA: the Q tile once, then per block of 128 keys the K tile (a
+//            three-stage ring, released once S_j = Q K_j^T is done) and the
+//            V^T tile with the key scales (a two-stage ring, released once
+//            P_j V_j is done);
 //   warp 1   tensor memory (512 columns: two 128-column score buffers and the
 //            128-column output accumulator O); one lane issues S_j = Q K_j^T
 //            (kind::i8, 128 x 128 x 128) into score buffer j % 2, then
 //            O += P_{j-1} V_{j-1} (kind::f16, bf16 in, fp32 accumulation),
 //            so S_j is computed while the softmax works on block j-1;
-//   warps 2-9 softmax, two threads per query row (tensor-memory lane), each
-//            with 64 keys of the block: reads its half score row, scales it
-//            with the key scales (staged in shared memory with the K tile),
-//            exchanges the half-row maxima, keeps a running maximum m and sum l
-//            (fp32, of the unrounded weights), writes P = 2^(s - m) as bf16 into
-//            its 128-byte swizzled half-tile, and at the end writes its half of
-//            O / l as bf16.
+//   warps 2-17 softmax, four threads per query row (tensor-memory lane), each
+//            with 32 keys of the block: reads its score slice, scales it with
+//            the key scales, exchanges the part-row maxima through shared
+//            memory and a bounded mbarrier, keeps a running maximum m and sum l
+//            (fp32, of the unrounded weights), writes P = 2^(s - m) as bf16
+//            into its four 16-byte chunks of the 128-byte swizzled P tile
+//            (double-buffered), and at the end writes its 32 columns of O / l.
 //            The maximum used for the exponent is raised only when a row's
 //            maximum grows by more than 2^8 (P stays below 256); O is then
 //            rescaled in tensor memory after the previous P.V has completed.
@@ -46,12 +48,14 @@ constexpr int kAttQBytes = 128 * 128;      // int8 Q tile
 constexpr int kAttKBytes = 128 * 128;      // int8 K tile
 constexpr int kAttVBytes = 2 * 128 * 128;  // bf16 V^T tile (128 d rows x 128 keys), two 64-key boxes
 constexpr int kAttPBytes = 2 * 128 * 128;  // bf16 P tile (128 rows x 128 keys), two 64-key halves
-constexpr int kAttStages = 2;
-constexpr int kAttThreads = 320;  // producer, MMA, 8 softmax warps (two threads per query row)
+constexpr int kAttKStages = 3;  // K ring: K_{j+3} loads once S_j = Q K_j^T is done
+constexpr int kAttVStages = 2;  // V^T ring (with the key scales): V_{j+2} loads once P_j V_j is done
+constexpr int kAttParts = 4;      // softmax threads per query row (32 keys of a block each)
+constexpr int kAttThreads = 64 + 128 * kAttParts;  // producer, MMA, 16 softmax warps
 constexpr int kAttKsBytes = 128 * 4;  // the key block's scales
-constexpr size_t kAttSmem = size_t(kAttQBytes) + kAttStages * (kAttKBytes + kAttVBytes + kAttKsBytes) +
-                            2 * kAttPBytes + 2 * 2 * 128 * 4 /*row max exchange*/ + 2 * 128 * 4 /*row sums*/ +
-                            1024 + 256;
+constexpr size_t kAttSmem = size_t(kAttQBytes) + kAttKStages * kAttKBytes + kAttVStages * (kAttVBytes + kAttKsBytes) +
+                            2 * kAttPBytes + 2 * kAttParts * 128 * 4 /*row max exchange*/ +
+                            kAttParts * 128 * 4 /*row sums*/ + 1024 + 256;
 
 struct AttParams {
   int S, H;
@@ -174,24 +178,26 @@ __global__ void __launch_bounds__(kAttThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kAttQBytes;                   // [stage][128 keys x 128 B]
-  uint8_t* sV = sK + kAttStages * kAttKBytes;      // [stage][2 boxes: 128 d rows x 64 keys (128 B)]
-  uint8_t* sP = sV + kAttStages * kAttVBytes;      // [buffer][2 halves: 128 rows x 64 keys (128 B)]
-  float* sKs = reinterpret_cast<float*>(sP + 2 * kAttPBytes);  // [stage][128] key scales
-  float* xmax = sKs + kAttStages * 128;            // [block parity][half][128 rows]: half-row maxima
-  float* xsum = xmax + 2 * 2 * 128;                // [half][128 rows]: half-row sums at the end
-  uint64_t* bars = reinterpret_cast<uint64_t*>(xsum + 2 * 128);
+  uint8_t* sK = sQ + kAttQBytes;                   // [K stage][128 keys x 128 B]
+  uint8_t* sV = sK + kAttKStages * kAttKBytes;     // [V stage][2 boxes: 128 d rows x 64 keys (128 B)]
+  uint8_t* sP = sV + kAttVStages * kAttVBytes;     // [buffer][2 halves: 128 rows x 64 keys (128 B)]
+  float* sKs = reinterpret_cast<float*>(sP + 2 * kAttPBytes);  // [V stage][128] key scales
+  float* xmax = sKs + kAttVStages * 128;           // [block parity][part][128 rows]: part-row maxima
+  float* xsum = xmax + 2 * kAttParts * 128;        // [part][128 rows]: part-row sums at the end
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xsum + kAttParts * 128);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_empty = bars + 7;   // [2]
-  uint64_t* p_full = bars + 9;    // [2]
-  uint64_t* pv_done = bars + 11;  // [2]
-  uint64_t* drain = bars + 13;
-  uint64_t* xchg = bars + 14;     // [2]: the 256 softmax threads exchanged their half-row maxima
-  uint64_t* xsum_bar = bars + 16; // the 256 softmax threads stored their half-row sums
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* k_full = bars + 1;    // [K stage]
+  uint64_t* k_empty = bars + 4;   // [K stage]
+  uint64_t* v_full = bars + 7;    // [V stage]: V^T and the key scales
+  uint64_t* v_empty = bars + 9;   // [V stage]
+  uint64_t* s_full = bars + 11;   // [2]
+  uint64_t* s_empty = bars + 13;  // [2]
+  uint64_t* p_full = bars + 15;   // [2]
+  uint64_t* pv_done = bars + 17;  // [2]
+  uint64_t* drain = bars + 19;
+  uint64_t* xchg = bars + 20;     // [2]: the softmax threads exchanged their part-row maxima
+  uint64_t* xsum_bar = bars + 22; // the softmax threads stored their part-row sums
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -202,17 +208,23 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    for (int st = 0; st < kAttKStages; ++st) {
+      mbar_init(&k_full[st], 1);
+      mbar_init(&k_empty[st], 1);
+    }
+    for (int st = 0; st < kAttVStages; ++st) {
+      mbar_init(&v_full[st], 1);
+      mbar_init(&v_empty[st], 1);
+    }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&kv_full[b], 1);
-      mbar_init(&kv_empty[b], 1);
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 8);
-      mbar_init(&p_full[b], 8);
+      mbar_init(&s_empty[b], 4 * kAttParts);
+      mbar_init(&p_full[b], 4 * kAttParts);
       mbar_init(&pv_done[b], 1);
-      mbar_init(&xchg[b], 256);
+      mbar_init(&xchg[b], 128 * kAttParts);
     }
     mbar_init(drain, 1);
-    mbar_init(xsum_bar, 256);
+    mbar_init(xsum_bar, 128 * kAttParts);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -233,14 +245,20 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       mbar_arrive_expect_tx(q_full, kAttQBytes);
       tma_load_2d(sQ, &tmQ, q_full, 0, h * S + qb * kAttBlk, pol_q);
       for (int j = 0; j < nb; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait_bounded(&kv_empty[st], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), limit, abort_flag)) break;
+        const int kst = j % kAttKStages, vst = j % kAttVStages;
+        if (!mbar_wait_bounded(&k_empty[kst], static_cast<uint32_t>(((j / kAttKStages) & 1) ^ 1), limit,
+                               abort_flag))
+          break;
+        mbar_arrive_expect_tx(&k_full[kst], kAttKBytes);
+        tma_load_2d(sK + kst * kAttKBytes, &tmK, &k_full[kst], 0, h * S + j * kAttBlk, pol_kv);
+        if (!mbar_wait_bounded(&v_empty[vst], static_cast<uint32_t>(((j / kAttVStages) & 1) ^ 1), limit,
+                               abort_flag))
+          break;
         const uint32_t ks_bytes = static_cast<uint32_t>(min(kAttBlk, S - j * kAttBlk) * 4);  // S % 8 == 0
-        mbar_arrive_expect_tx(&kv_full[st], kAttKBytes + kAttVBytes + ks_bytes);
-        bulk_load(sKs + st * 128, p.ks + int64_t(h) * S + j * kAttBlk, ks_bytes, &kv_full[st], pol_kv);
-        tma_load_2d(sK + st * kAttKBytes, &tmK, &kv_full[st], 0, h * S + j * kAttBlk, pol_kv);
-        tma_load_2d(sV + st * kAttVBytes, &tmV, &kv_full[st], j * kAttBlk, h * kAttD, pol_kv);
-        tma_load_2d(sV + st * kAttVBytes + kAttVBytes / 2, &tmV, &kv_full[st], j * kAttBlk + 64, h * kAttD, pol_kv);
+        mbar_arrive_expect_tx(&v_full[vst], kAttVBytes + ks_bytes);
+        bulk_load(sKs + vst * 128, p.ks + int64_t(h) * S + j * kAttBlk, ks_bytes, &v_full[vst], pol_kv);
+        tma_load_2d(sV + vst * kAttVBytes, &tmV, &v_full[vst], j * kAttBlk, h * kAttD, pol_kv);
+        tma_load_2d(sV + vst * kAttVBytes + kAttVBytes / 2, &tmV, &v_full[vst], j * kAttBlk + 64, h * kAttD, pol_kv);
       }
     }
   } else if (warp == 1) {
@@ -252,21 +270,23 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       const uint64_t qd = smem_desc_sw128(smem_u32(sQ));
       for (int j = 0; ok && j <= nb; ++j) {
         if (j < nb) {  // S_j = Q K_j^T into score buffer j % 2
-          const int st = j & 1;
-          if (!mbar_wait_bounded(&kv_full[st], static_cast<uint32_t>((j >> 1) & 1), limit, abort_flag) ||
-              !mbar_wait_bounded(&s_empty[st], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), limit, abort_flag)) {
+          const int st = j % kAttKStages, b = j & 1;
+          if (!mbar_wait_bounded(&k_full[st], static_cast<uint32_t>((j / kAttKStages) & 1), limit, abort_flag) ||
+              !mbar_wait_bounded(&s_empty[b], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), limit, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t kd = smem_desc_sw128(smem_u32(sK + st * kAttKBytes));
 #pragma unroll
-          for (int k = 0; k < 4; ++k) mma_i8(tmem + st * kAttBlk, qd + 2u * k, kd + 2u * k, idesc_s, k > 0 ? 1u : 0u);
-          mma_commit(&s_full[st]);
+          for (int k = 0; k < 4; ++k) mma_i8(tmem + b * kAttBlk, qd + 2u * k, kd + 2u * k, idesc_s, k > 0 ? 1u : 0u);
+          mma_commit(&s_full[b]);
+          mma_commit(&k_empty[st]);
         }
         if (j >= 1) {  // O += P_{j-1} V_{j-1}
-          const int t = j - 1, bt = t & 1;
-          if (!mbar_wait_bounded(&p_full[bt], static_cast<uint32_t>((t >> 1) & 1), limit, abort_flag)) {
+          const int t = j - 1, bt = t & 1, stt = t % kAttVStages;
+          if (!mbar_wait_bounded(&v_full[stt], static_cast<uint32_t>((t / kAttVStages) & 1), limit, abort_flag) ||
+              !mbar_wait_bounded(&p_full[bt], static_cast<uint32_t>((t >> 1) & 1), limit, abort_flag)) {
             ok = false;
             break;
           }
@@ -275,27 +295,28 @@ __global__ void __launch_bounds__(kAttThreads, 1)
           for (int k = 0; k < 8; ++k) {  // 16 keys = 32 bytes per K step; halves of 64 keys
             const int half = k >> 2;
             const uint64_t pd = smem_desc_sw128(smem_u32(sP + bt * kAttPBytes + half * (kAttPBytes / 2)));
-            const uint64_t vd = smem_desc_sw128(smem_u32(sV + bt * kAttVBytes + half * (kAttVBytes / 2)));
+            const uint64_t vd = smem_desc_sw128(smem_u32(sV + stt * kAttVBytes + half * (kAttVBytes / 2)));
             mma_bf16(tmem + 2 * kAttBlk, pd + 2u * (k & 3), vd + 2u * (k & 3), idesc_o, (t > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit(&pv_done[bt]);
-          mma_commit(&kv_empty[bt]);
+          mma_commit(&v_empty[stt]);
         }
       }
       mma_commit(drain);
       mbar_wait_bounded(drain, 0, limit, nullptr);
     }
   } else {
-    // -------------------------------------------------------------- softmax (warps 2..9)
-    // Two threads per query row (TMEM lane): warps 2-5 take keys [0, 64) of each
-    // block and columns [0, 64) of O, warps 6-9 keys [64, 128) and columns [64, 128).
-    // The two halves exchange their row maxima through shared memory and a
-    // 256-arrival mbarrier per block, so both take the same rescale decisions.
+    // -------------------------------------------------------------- softmax (warps 2..17)
+    // Four threads per query row (TMEM lane): part q = (warp - 2) / 4 takes keys
+    // [32 q, 32 q + 32) of each block and columns [32 q, 32 q + 32) of O. The parts
+    // exchange their row maxima through shared memory and a bounded mbarrier per
+    // block, so all four take the same rescale decisions.
     const int quarter = warp & 3;                     // TMEM lanes 32*quarter .. +31
-    const int half = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;                // query row within the block
     const int i = qb * kAttBlk + r;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t o_cols = tmem + lane_base + 2 * kAttBlk + 32 * part;
     const float cq = __fmul_rn(i < S ? __ldg(p.qs + int64_t(h) * S + i) : 0.0f, p.c);
     float m_used = -INFINITY;
     float2 l2 = make_float2(0.0f, 0.0f);  // running sum of the weights, two partial sums
@@ -304,12 +325,11 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       return __all_sync(0xFFFFFFFFu, mbar_wait_bounded(bar, parity, limit, abort_flag));
     };
     for (int j = 0; j < nb; ++j) {
-      const int b = j & 1, st = j & 1;
+      const int b = j & 1, st = j % kAttVStages;
       if (!(ok = wait_all(&s_full[b], static_cast<uint32_t>((j >> 1) & 1)))) break;
       tc_fence_after();
-      uint32_t sr[2][32];
-#pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) tmem_ld32(tmem + lane_base + b * kAttBlk + 64 * half + 32 * c2, sr[c2]);
+      uint32_t sr[32];
+      tmem_ld32(tmem + lane_base + b * kAttBlk + 32 * part, sr);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -318,32 +338,31 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       // acc + 1.5 * 2^23 read as a float, minus 1.5 * 2^23, are (float)acc without the
       // conversion unit); the log2-domain score is s' * cq, cq = qs_i log2(e) / sqrt(128) >= 0,
       // so maxima can be taken on s'. Keys past the end (last block only) are masked.
-      const int key0 = j * kAttBlk + 64 * half;
-      const bool partial = key0 + 64 > S;
-      const float* ksb = sKs + st * 128 + 64 * half;
+      const int key0 = j * kAttBlk + 32 * part;
+      const bool partial = key0 + 32 > S;
+      // the key scales travel with V_j (that stage is released only after P_j V_j)
+      if (!(ok = wait_all(&v_full[st], static_cast<uint32_t>((j / kAttVStages) & 1)))) break;
+      const float* ksb = sKs + st * 128 + 32 * part;
       float mx = -INFINITY;
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
+      for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 kv = *reinterpret_cast<const float4*>(ksb + 4 * e4);
+        const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+        float sc[4];
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 kv = *reinterpret_cast<const float4*>(ksb + 32 * c2 + 4 * e4);
-          const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
-          float sc[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * e4 + e;
-            sc[e] = __fmul_rn(__fsub_rn(__uint_as_float(sr[c2][c] + 0x4B400000u), 12582912.0f), kk[e]);
-            if (partial && key0 + 32 * c2 + c >= S) sc[e] = -INFINITY;
-            sr[c2][c] = __float_as_uint(sc[e]);
-          }
-          mx = att_max3(mx, att_max3(sc[0], sc[1], sc[2]), sc[3]);
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * e4 + e;
+          sc[e] = __fmul_rn(__fsub_rn(__uint_as_float(sr[c] + 0x4B400000u), 12582912.0f), kk[e]);
+          if (partial && key0 + c >= S) sc[e] = -INFINITY;
+          sr[c] = __float_as_uint(sc[e]);
         }
+        mx = att_max3(mx, att_max3(sc[0], sc[1], sc[2]), sc[3]);
       }
-      float* xm = xmax + b * 256;
-      xm[half * 128 + r] = mx;
+      float* xm = xmax + b * (kAttParts * 128);
+      xm[part * 128 + r] = mx;
       mbar_arrive(&xchg[b]);
       if (!(ok = wait_all(&xchg[b], static_cast<uint32_t>((j >> 1) & 1)))) break;
-      mx = fmaxf(mx, xm[(1 - half) * 128 + r]);
+      mx = att_max3(att_max3(xm[r], xm[128 + r], xm[256 + r]), xm[384 + r], -INFINITY);
       // raise the exponent's maximum when the row maximum grew by more than 2^8 (log2 units)
       const bool need = j == 0 || __fmul_rn(mx - m_used, cq) > 8.0f;
       if (__ballot_sync(0xFFFFFFFFu, need) != 0u && j > 0) {
@@ -351,16 +370,12 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         if (!(ok = wait_all(&pv_done[(j - 1) & 1], static_cast<uint32_t>(((j - 1) >> 1) & 1)))) break;
         tc_fence_after();
         const float f = need ? ex2_approx(__fmul_rn(m_used - mx, cq)) : 1.0f;
-#pragma unroll 1
-        for (int c2 = 0; c2 < 2; ++c2) {
-          uint32_t o[32];
-          const uint32_t oaddr = tmem + lane_base + 2 * kAttBlk + 64 * half + 32 * c2;
-          tmem_ld32(oaddr, o);
-          tmem_ld_wait();
+        uint32_t o[32];
+        tmem_ld32(o_cols, o);
+        tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), f));
-          tmem_st32(oaddr, o);
-        }
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), f));
+        tmem_st32(o_cols, o);
         tmem_st_wait();
         l2 = __fmul2_rn(l2, make_float2(f, f));
       }
@@ -368,18 +383,18 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       if (j >= 2) {  // P buffer b was last read by P_{j-2} V_{j-2}
         if (!(ok = wait_all(&pv_done[b], static_cast<uint32_t>(((j - 2) >> 1) & 1)))) break;
       }
-      // P = 2^(s' cq - m cq) as bf16 into row r of the half-tile (16-byte chunk c at
-      // position c ^ (r % 8) of the 128-byte row); l sums the weights in fp32, in pairs
+      // P = 2^(s' cq - m cq) as bf16: this part's 32 keys are chunks 4 (part % 2) .. +3 of row r
+      // of half-tile part / 2 (16-byte chunk c at position c ^ (r % 8) of the 128-byte row)
       const float nm = -__fmul_rn(m_used, cq);
-      uint8_t* prow = sP + b * kAttPBytes + half * (kAttPBytes / 2) + r * 128;
+      uint8_t* prow = sP + b * kAttPBytes + (part >> 1) * (kAttPBytes / 2) + r * 128;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int c0 = 8 * ch + 2 * e;
-          float p0 = ex2_approx(__fmaf_rn(__uint_as_float(sr[c0 >> 5][c0 & 31]), cq, nm));
-          float p1 = ex2_approx(__fmaf_rn(__uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]), cq, nm));
+          const int c0 = 8 * cc + 2 * e;
+          float p0 = ex2_approx(__fmaf_rn(__uint_as_float(sr[c0]), cq, nm));
+          float p1 = ex2_approx(__fmaf_rn(__uint_as_float(sr[c0 + 1]), cq, nm));
           if (partial) {  // masked keys weigh 0 (also when cq = 0, where -inf * cq is not a number)
             if (key0 + c0 >= S) p0 = 0.0f;
             if (key0 + c0 + 1 >= S) p1 = 0.0f;
@@ -387,6 +402,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
           w[e] = pack_bf16x2(p0, p1);
           l2 = __fadd2_rn(l2, make_float2(p0, p1));
         }
+        const int ch = 4 * (part & 1) + cc;
         *reinterpret_cast<uint4*>(prow + 16 * (ch ^ (r & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();  // the tensor core reads P through the async proxy
@@ -399,29 +415,27 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       ok = wait_all(&pv_done[t & 1], static_cast<uint32_t>((t >> 1) & 1));
     }
     if (ok) {
-      xsum[half * 128 + r] = __fadd_rn(l2.x, l2.y);
+      xsum[part * 128 + r] = __fadd_rn(l2.x, l2.y);
       mbar_arrive(xsum_bar);
       ok = wait_all(xsum_bar, 0);
     }
     if (ok) {
       tc_fence_after();
-      const float inv_l = __fdiv_rn(1.0f, __fadd_rn(xsum[r], xsum[128 + r]));
-      __nv_bfloat16* orow = p.out + int64_t(i) * p.ld_out + h * kAttD + 64 * half;
-#pragma unroll 1
-      for (int c2 = 0; c2 < 2; ++c2) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_base + 2 * kAttBlk + 64 * half + 32 * c2, o);
-        tmem_ld_wait();
-        if (i < S) {
+      const float lsum = __fadd_rn(__fadd_rn(xsum[r], xsum[128 + r]), __fadd_rn(xsum[256 + r], xsum[384 + r]));
+      const float inv_l = __fdiv_rn(1.0f, lsum);
+      __nv_bfloat16* orow = p.out + int64_t(i) * p.ld_out + h * kAttD + 32 * part;
+      uint32_t o[32];
+      tmem_ld32(o_cols, o);
+      tmem_ld_wait();
+      if (i < S) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            uint32_t w[4];
+        for (int g = 0; g < 4; ++g) {
+          uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = pack_bf16x2(__fmul_rn(__uint_as_float(o[8 * g + 2 * e]), inv_l),
-                                 __fmul_rn(__uint_as_float(o[8 * g + 2 * e + 1]), inv_l));
-            *reinterpret_cast<uint4*>(orow + 32 * c2 + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+          for (int e = 0; e < 4; ++e)
+            w[e] = pack_bf16x2(__fmul_rn(__uint_as_float(o[8 * g + 2 * e]), inv_l),
+                               __fmul_rn(__uint_as_float(o[8 * g + 2 * e + 1]), inv_l));
+          *reinterpret_cast<uint4*>(orow + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
