@@ -13,23 +13,28 @@
 // attn_kernel: one CTA per (head, 128-query block); warp roles:
 //   warp 0   TMA: the Q tile once, then per block of 128 keys the K tile (a
 //            three-stage ring, released once S_j = Q K_j^T is done) and the
-//            V^T tile with the key scales (a two-stage ring, released once
+//            V^T tile with the key scales (a three-stage ring, released once
 //            P_j V_j is done);
-//   warp 1   tensor memory (512 columns: two 128-column score buffers and the
-//            128-column output accumulator O); one lane issues S_j = Q K_j^T
-//            (kind::i8, 128 x 128 x 128) into score buffer j % 2, then
-//            O += P_{j-1} V_{j-1} (kind::f16, bf16 in, fp32 accumulation),
-//            so S_j is computed while the softmax works on block j-1;
-//   warps 2-17 softmax, four threads per query row (tensor-memory lane), each
-//            with 32 keys of the block: reads its score slice, scales it with
-//            the key scales, exchanges the part-row maxima through shared
-//            memory and a bounded mbarrier, keeps a running maximum m and sum l
-//            (fp32, of the unrounded weights), writes P = 2^(s - m) as bf16
-//            into its four 16-byte chunks of the 128-byte swizzled P tile
-//            (double-buffered), and at the end writes its 32 columns of O / l.
-//            The maximum used for the exponent is raised only when a row's
-//            maximum grows by more than 2^8 (P stays below 256); O is then
-//            rescaled in tensor memory after the previous P.V has completed.
+//   warp 1   tensor memory (512 columns: two 128-column score buffers, the
+//            128-column output accumulator O and two 64-column P buffers);
+//            one lane issues S_j = Q K_j^T (kind::i8, 128 x 128 x 128) into
+//            score buffer j % 2 as soon as block j-2's scores have been read,
+//            and O += P_j V_j (kind::f16, A = P_j from tensor memory, B = V_j^T
+//            from shared memory, fp32 accumulation) once P_j is written;
+//   warps 2-3 idle;
+//   warps 4-11 softmax, two sets of four warps, one thread per query row
+//            (tensor-memory lane): set 0 takes the even key blocks, set 1 the
+//            odd ones, so one set's exponentials overlap the other's score
+//            loads. For its block a thread reads the whole score row, scales
+//            it with the key scales, takes the row maximum, and writes
+//            P = 2^(s - m) as bf16 into P buffer j % 2. The maximum m used in
+//            the exponent is handed from block to block through shared memory
+//            (the set of block j publishes it, the set of block j+1 waits for
+//            it); it is raised only when a row's maximum grows by more than
+//            2^8 (P stays below 256), and O is then rescaled in tensor memory
+//            after P_{j-1} V_{j-1} has completed. Each set keeps the sum of its
+//            own weights; at the end the two sums are added, and set s writes
+//            columns [64 s, 64 s + 64) of O / l.
 // Every wait is bounded (the kernel records a timeout and drains).
 #pragma once
 
@@ -47,15 +52,23 @@ constexpr int kAttBlk = 128;               // queries per CTA, keys per block
 constexpr int kAttQBytes = 128 * 128;      // int8 Q tile
 constexpr int kAttKBytes = 128 * 128;      // int8 K tile
 constexpr int kAttVBytes = 2 * 128 * 128;  // bf16 V^T tile (128 d rows x 128 keys), two 64-key boxes
-constexpr int kAttPBytes = 2 * 128 * 128;  // bf16 P tile (128 rows x 128 keys), two 64-key halves
 constexpr int kAttKStages = 3;  // K ring: K_{j+3} loads once S_j = Q K_j^T is done
-constexpr int kAttVStages = 2;  // V^T ring (with the key scales): V_{j+2} loads once P_j V_j is done
-constexpr int kAttParts = 4;      // softmax threads per query row (32 keys of a block each)
-constexpr int kAttThreads = 64 + 128 * kAttParts;  // producer, MMA, 16 softmax warps
-constexpr int kAttKsBytes = 128 * 4;  // the key block's scales
-constexpr size_t kAttSmem = size_t(kAttQBytes) + kAttKStages * kAttKBytes + kAttVStages * (kAttVBytes + kAttKsBytes) +
-                            2 * kAttPBytes + 2 * kAttParts * 128 * 4 /*row max exchange*/ +
-                            kAttParts * 128 * 4 /*row sums*/ + 1024 + 256;
+constexpr int kAttVStages = 3;  // V^T ring (with the key scales): V_{j+3} loads once P_j V_j is done
+constexpr int kAttThreads = 128 + 2 * 128;  // producer, MMA (and two idle warps), two softmax sets
+// Register split (setmaxnreg): the first warpgroup gives registers back, the two
+// softmax warpgroups take them. The kernel is launched with at least
+// kAttRegsLaunch registers per thread (the host checks the compiled count), so
+// the split never asks for more than the block holds.
+constexpr uint32_t kAttRegsCtl = 40, kAttRegsSoftmax = 232, kAttRegsLaunch = 168;
+static_assert(128 * kAttRegsCtl + 256 * kAttRegsSoftmax <= kAttThreads * kAttRegsLaunch, "register split");
+constexpr int kAttKsBytes = 128 * 4;       // the key block's scales
+// tensor-memory columns
+constexpr uint32_t kAttColS = 0;    // score buffers b at b * 128 (int32)
+constexpr uint32_t kAttColO = 256;  // output accumulator (fp32)
+constexpr uint32_t kAttColP = 384;  // P buffers b at 384 + b * 64 (bf16 pairs)
+constexpr size_t kAttSmem = size_t(kAttQBytes) + kAttKStages * kAttKBytes +
+                            kAttVStages * (size_t(kAttVBytes) + kAttKsBytes) + 2 * 128 * 4 /*maxima*/ +
+                            2 * 128 * 4 /*row sums*/ + 1024 + 256;
 
 struct AttParams {
   int S, H;
@@ -81,14 +94,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32, one CTA.
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 x bf16 -> fp32, one CTA. A (M = 128
+// rows in lanes 0-127) holds two bf16 per 32-bit column, the lower-indexed K
+// element in the low half; one instruction reads 16 K elements (8 columns).
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -108,10 +123,83 @@ __device__ __forceinline__ float att_max3(float a, float b, float c) {
   return r;
 }
 
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Scales a block's raw scores in place, s'_k = (float)acc_k * ks_k, and returns
+// their maximum. |acc| <= 127^2 * 128 < 2^22, so the bits of acc + 1.5 * 2^23
+// read as a float, minus 1.5 * 2^23, are (float)acc exactly, without the
+// conversion unit. With kMasked, keys k >= nvalid (past the end of the
+// sequence) get s' = -inf; the two forms are separate so the unmasked one,
+// used for every block but the last, carries no per-key predicates.
+template <bool kMasked>
+__device__ __forceinline__ float att_scores(uint32_t (&sr)[4][32], const float* ksb, int nvalid) {
+  const float2 magic2 = make_float2(-12582912.0f, -12582912.0f);
+  float mx = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+#pragma unroll
+    for (int e4 = 0; e4 < 8; ++e4) {
+      const int k0 = 4 * e4;
+      const float4 kv = *reinterpret_cast<const float4*>(ksb + 32 * c + k0);
+      float2 x01 = make_float2(__uint_as_float(sr[c][k0] + 0x4B400000u), __uint_as_float(sr[c][k0 + 1] + 0x4B400000u));
+      float2 x23 =
+          make_float2(__uint_as_float(sr[c][k0 + 2] + 0x4B400000u), __uint_as_float(sr[c][k0 + 3] + 0x4B400000u));
+      x01 = __fmul2_rn(__fadd2_rn(x01, magic2), make_float2(kv.x, kv.y));
+      x23 = __fmul2_rn(__fadd2_rn(x23, magic2), make_float2(kv.z, kv.w));
+      float sc[4] = {x01.x, x01.y, x23.x, x23.y};
+      if (kMasked) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (32 * c + k0 + e >= nvalid) sc[e] = -INFINITY;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sr[c][k0 + e] = __float_as_uint(sc[e]);
+      mx = att_max3(mx, att_max3(sc[0], sc[1], sc[2]), sc[3]);
+    }
+  }
+  return mx;
+}
+
+// P_k = 2^(s'_k cq - m cq) as bf16 pairs (lower key in the low half) into the
+// 64 P columns at p_cols; returns the sum of the (unrounded) weights. With
+// kMasked, keys k >= nvalid weigh 0 (also when cq = 0, where -inf * cq is not a
+// number).
+template <bool kMasked>
+__device__ __forceinline__ float2 att_weights(const uint32_t (&sr)[4][32], float2 cq2, float2 nm2, int nvalid,
+                                              uint32_t p_cols) {
+  float2 bs2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    uint32_t w[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int k0 = 64 * hh + 2 * e;
+      const float2 t = __ffma2_rn(
+          make_float2(__uint_as_float(sr[k0 >> 5][k0 & 31]), __uint_as_float(sr[k0 >> 5][(k0 & 31) + 1])), cq2, nm2);
+      float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
+      if (kMasked) {
+        if (k0 >= nvalid) p0 = 0.0f;
+        if (k0 + 1 >= nvalid) p1 = 0.0f;
+      }
+      w[e] = pack_bf16x2(p0, p1);
+      bs2 = __fadd2_rn(bs2, make_float2(p0, p1));
+    }
+    tmem_st32(p_cols + 32 * hh, w);
+  }
+  return bs2;
 }
 
 // ---------------------------------------------------------------- prep
@@ -180,24 +268,23 @@ __global__ void __launch_bounds__(kAttThreads, 1)
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + kAttQBytes;                   // [K stage][128 keys x 128 B]
   uint8_t* sV = sK + kAttKStages * kAttKBytes;     // [V stage][2 boxes: 128 d rows x 64 keys (128 B)]
-  uint8_t* sP = sV + kAttVStages * kAttVBytes;     // [buffer][2 halves: 128 rows x 64 keys (128 B)]
-  float* sKs = reinterpret_cast<float*>(sP + 2 * kAttPBytes);  // [V stage][128] key scales
-  float* xmax = sKs + kAttVStages * 128;           // [block parity][part][128 rows]: part-row maxima
-  float* xsum = xmax + 2 * kAttParts * 128;        // [part][128 rows]: part-row sums at the end
-  uint64_t* bars = reinterpret_cast<uint64_t*>(xsum + kAttParts * 128);
+  float* sKs = reinterpret_cast<float*>(sV + kAttVStages * kAttVBytes);  // [V stage][128] key scales
+  float* sMx = sKs + kAttVStages * 128;            // [block parity][128 rows]: the maximum after a block
+  float* sL = sMx + 2 * 128;                       // [set][128 rows]: the sets' row sums at the end
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sL + 2 * 128);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;    // [K stage]
   uint64_t* k_empty = bars + 4;   // [K stage]
   uint64_t* v_full = bars + 7;    // [V stage]: V^T and the key scales
-  uint64_t* v_empty = bars + 9;   // [V stage]
-  uint64_t* s_full = bars + 11;   // [2]
-  uint64_t* s_empty = bars + 13;  // [2]
-  uint64_t* p_full = bars + 15;   // [2]
-  uint64_t* pv_done = bars + 17;  // [2]
-  uint64_t* drain = bars + 19;
-  uint64_t* xchg = bars + 20;     // [2]: the softmax threads exchanged their part-row maxima
-  uint64_t* xsum_bar = bars + 22; // the softmax threads stored their part-row sums
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
+  uint64_t* v_empty = bars + 10;  // [V stage]
+  uint64_t* s_full = bars + 13;   // [score buffer]
+  uint64_t* s_empty = bars + 15;  // [score buffer]: its scores are in the softmax threads' registers
+  uint64_t* p_full = bars + 17;   // [P buffer]
+  uint64_t* pv_done = bars + 19;  // [P buffer]: P_j V_j has completed
+  uint64_t* mx_full = bars + 21;  // [block parity]: the maximum after the block is published
+  uint64_t* l_full = bars + 23;   // both sets stored their row sums
+  uint64_t* drain = bars + 24;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 25);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -218,13 +305,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 4 * kAttParts);
-      mbar_init(&p_full[b], 4 * kAttParts);
+      mbar_init(&s_empty[b], 4);   // one arrival per warp of the set
+      mbar_init(&p_full[b], 4);
       mbar_init(&pv_done[b], 1);
-      mbar_init(&xchg[b], 128 * kAttParts);
+      mbar_init(&mx_full[b], 4);
     }
+    mbar_init(l_full, 8);
     mbar_init(drain, 1);
-    mbar_init(xsum_bar, 128 * kAttParts);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -237,205 +324,207 @@ __global__ void __launch_bounds__(kAttThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ producer
-      const uint64_t pol_q = policy_evict_first();
-      const uint64_t pol_kv = policy_evict_last();  // every query block of the head re-reads K and V
-      mbar_arrive_expect_tx(q_full, kAttQBytes);
-      tma_load_2d(sQ, &tmQ, q_full, 0, h * S + qb * kAttBlk, pol_q);
-      for (int j = 0; j < nb; ++j) {
-        const int kst = j % kAttKStages, vst = j % kAttVStages;
-        if (!mbar_wait_bounded(&k_empty[kst], static_cast<uint32_t>(((j / kAttKStages) & 1) ^ 1), limit,
-                               abort_flag))
-          break;
-        mbar_arrive_expect_tx(&k_full[kst], kAttKBytes);
-        tma_load_2d(sK + kst * kAttKBytes, &tmK, &k_full[kst], 0, h * S + j * kAttBlk, pol_kv);
-        if (!mbar_wait_bounded(&v_empty[vst], static_cast<uint32_t>(((j / kAttVStages) & 1) ^ 1), limit,
-                               abort_flag))
-          break;
-        const uint32_t ks_bytes = static_cast<uint32_t>(min(kAttBlk, S - j * kAttBlk) * 4);  // S % 8 == 0
-        mbar_arrive_expect_tx(&v_full[vst], kAttVBytes + ks_bytes);
-        bulk_load(sKs + vst * 128, p.ks + int64_t(h) * S + j * kAttBlk, ks_bytes, &v_full[vst], pol_kv);
-        tma_load_2d(sV + vst * kAttVBytes, &tmV, &v_full[vst], j * kAttBlk, h * kAttD, pol_kv);
-        tma_load_2d(sV + vst * kAttVBytes + kAttVBytes / 2, &tmV, &v_full[vst], j * kAttBlk + 64, h * kAttD, pol_kv);
+  if (warp < 4) {
+    regs_dec<kAttRegsCtl>();  // inside the role's branch: the compiler's register limit follows it
+    if (warp == 0) {
+      if (lane == 0) {
+        // ------------------------------------------------------------ producer
+        const uint64_t pol_q = policy_evict_first();
+        const uint64_t pol_kv = policy_evict_last();  // every query block of the head re-reads K and V
+        mbar_arrive_expect_tx(q_full, kAttQBytes);
+        tma_load_2d(sQ, &tmQ, q_full, 0, h * S + qb * kAttBlk, pol_q);
+        int nk = 0, nv = 0;  // loads issued
+        for (int j = 0; j < nb; ++j) {
+          const int kst = j % kAttKStages, vst = j % kAttVStages;
+          if (!mbar_wait_bounded(&k_empty[kst], static_cast<uint32_t>(((j / kAttKStages) & 1) ^ 1), limit,
+                                 abort_flag))
+            break;
+          mbar_arrive_expect_tx(&k_full[kst], kAttKBytes);
+          tma_load_2d(sK + kst * kAttKBytes, &tmK, &k_full[kst], 0, h * S + j * kAttBlk, pol_kv);
+          ++nk;
+          if (!mbar_wait_bounded(&v_empty[vst], static_cast<uint32_t>(((j / kAttVStages) & 1) ^ 1), limit,
+                                 abort_flag))
+            break;
+          const uint32_t ks_bytes = static_cast<uint32_t>(min(kAttBlk, S - j * kAttBlk) * 4);  // S % 8 == 0
+          mbar_arrive_expect_tx(&v_full[vst], kAttVBytes + ks_bytes);
+          bulk_load(sKs + vst * 128, p.ks + int64_t(h) * S + j * kAttBlk, ks_bytes, &v_full[vst], pol_kv);
+          tma_load_2d(sV + vst * kAttVBytes, &tmV, &v_full[vst], j * kAttBlk, h * kAttD, pol_kv);
+          tma_load_2d(sV + vst * kAttVBytes + kAttVBytes / 2, &tmV, &v_full[vst], j * kAttBlk + 64, h * kAttD, pol_kv);
+          ++nv;
+        }
+        // the copies still in flight land before the block exits (already done on the normal path)
+        mbar_wait_bounded(q_full, 0, limit, nullptr);
+        for (int t = max(0, nk - kAttKStages); t < nk; ++t)
+          mbar_wait_bounded(&k_full[t % kAttKStages], static_cast<uint32_t>((t / kAttKStages) & 1), limit, nullptr);
+        for (int t = max(0, nv - kAttVStages); t < nv; ++t)
+          mbar_wait_bounded(&v_full[t % kAttVStages], static_cast<uint32_t>((t / kAttVStages) & 1), limit, nullptr);
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc_s = idesc_i8(kAttBlk, kAttBlk);
-      constexpr uint32_t idesc_o = idesc_bf16(kAttBlk, kAttD);
-      bool ok = mbar_wait_bounded(q_full, 0, limit, abort_flag);
-      const uint64_t qd = smem_desc_sw128(smem_u32(sQ));
-      for (int j = 0; ok && j <= nb; ++j) {
-        if (j < nb) {  // S_j = Q K_j^T into score buffer j % 2
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        // Order: S_0, S_1, then per block t: S_{t+2} (once S_t has been read), O += P_t V_t.
+        constexpr uint32_t idesc_s = idesc_i8(kAttBlk, kAttBlk);
+        constexpr uint32_t idesc_o = idesc_bf16(kAttBlk, kAttD);
+        bool ok = mbar_wait_bounded(q_full, 0, limit, abort_flag);
+        const uint64_t qd = smem_desc_sw128(smem_u32(sQ));
+        auto issue_s = [&](int j) {  // S_j = Q K_j^T into score buffer j % 2
           const int st = j % kAttKStages, b = j & 1;
           if (!mbar_wait_bounded(&k_full[st], static_cast<uint32_t>((j / kAttKStages) & 1), limit, abort_flag) ||
-              !mbar_wait_bounded(&s_empty[b], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), limit, abort_flag)) {
-            ok = false;
-            break;
-          }
+              !mbar_wait_bounded(&s_empty[b], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), limit, abort_flag))
+            return false;
           tc_fence_after();
           const uint64_t kd = smem_desc_sw128(smem_u32(sK + st * kAttKBytes));
-#pragma unroll
-          for (int k = 0; k < 4; ++k) mma_i8(tmem + b * kAttBlk, qd + 2u * k, kd + 2u * k, idesc_s, k > 0 ? 1u : 0u);
+  #pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_i8(tmem + kAttColS + b * kAttBlk, qd + 2u * k, kd + 2u * k, idesc_s, k > 0 ? 1u : 0u);
           mma_commit(&s_full[b]);
           mma_commit(&k_empty[st]);
-        }
-        if (j >= 1) {  // O += P_{j-1} V_{j-1}
-          const int t = j - 1, bt = t & 1, stt = t % kAttVStages;
-          if (!mbar_wait_bounded(&v_full[stt], static_cast<uint32_t>((t / kAttVStages) & 1), limit, abort_flag) ||
+          return true;
+        };
+        for (int j = 0; ok && j < min(2, nb); ++j) ok = issue_s(j);
+        for (int t = 0; ok && t < nb; ++t) {
+          if (t + 2 < nb && !(ok = issue_s(t + 2))) break;
+          const int bt = t & 1, vst = t % kAttVStages;  // O += P_t V_t
+          if (!mbar_wait_bounded(&v_full[vst], static_cast<uint32_t>((t / kAttVStages) & 1), limit, abort_flag) ||
               !mbar_wait_bounded(&p_full[bt], static_cast<uint32_t>((t >> 1) & 1), limit, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {  // 16 keys = 32 bytes per K step; halves of 64 keys
+  #pragma unroll
+          for (int k = 0; k < 8; ++k) {  // 16 keys = 8 P columns = 32 bytes of a V^T row per K step
             const int half = k >> 2;
-            const uint64_t pd = smem_desc_sw128(smem_u32(sP + bt * kAttPBytes + half * (kAttPBytes / 2)));
-            const uint64_t vd = smem_desc_sw128(smem_u32(sV + stt * kAttVBytes + half * (kAttVBytes / 2)));
-            mma_bf16(tmem + 2 * kAttBlk, pd + 2u * (k & 3), vd + 2u * (k & 3), idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+            const uint64_t vd = smem_desc_sw128(smem_u32(sV + vst * kAttVBytes + half * (kAttVBytes / 2)));
+            mma_bf16_tmem_a(tmem + kAttColO, tmem + kAttColP + bt * 64 + 8 * k, vd + 2u * (k & 3), idesc_o,
+                            (t > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit(&pv_done[bt]);
-          mma_commit(&v_empty[stt]);
+          mma_commit(&v_empty[vst]);
         }
+        mma_commit(drain);
+        mbar_wait_bounded(drain, 0, limit, nullptr);
       }
-      mma_commit(drain);
-      mbar_wait_bounded(drain, 0, limit, nullptr);
     }
   } else {
-    // -------------------------------------------------------------- softmax (warps 2..17)
-    // Four threads per query row (TMEM lane): part q = (warp - 2) / 4 takes keys
-    // [32 q, 32 q + 32) of each block and columns [32 q, 32 q + 32) of O. The parts
-    // exchange their row maxima through shared memory and a bounded mbarrier per
-    // block, so all four take the same rescale decisions.
+    // -------------------------------------------------------------- softmax (warps 4..11)
+    regs_inc<kAttRegsSoftmax>();
+    const int set = (warp - 4) >> 2;                  // 0: even key blocks, 1: odd key blocks
     const int quarter = warp & 3;                     // TMEM lanes 32*quarter .. +31
-    const int part = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;                // query row within the block
     const int i = qb * kAttBlk + r;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t o_cols = tmem + lane_base + 2 * kAttBlk + 32 * part;
     const float cq = __fmul_rn(i < S ? __ldg(p.qs + int64_t(h) * S + i) : 0.0f, p.c);
-    float m_used = -INFINITY;
-    float2 l2 = make_float2(0.0f, 0.0f);  // running sum of the weights, two partial sums
+    float m_used = -INFINITY;             // the maximum this set's weights are relative to
+    float2 l2 = make_float2(0.0f, 0.0f);  // this set's sum of weights, two partial sums
     bool ok = true;
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xFFFFFFFFu, mbar_wait_bounded(bar, parity, limit, abort_flag));
     };
-    for (int j = 0; j < nb; ++j) {
-      const int b = j & 1, st = j % kAttVStages;
+    auto adopt = [&](float mp) {  // move this set's sum to the (larger) maximum mp
+      if (mp != m_used) {
+        if (m_used != -INFINITY) {
+          const float f = ex2_approx(__fmul_rn(m_used - mp, cq));
+          l2 = __fmul2_rn(l2, make_float2(f, f));
+        }
+        m_used = mp;
+      }
+    };
+    for (int j = set; j < nb; j += 2) {
+      const int b = j & 1, vst = j % kAttVStages;
       if (!(ok = wait_all(&s_full[b], static_cast<uint32_t>((j >> 1) & 1)))) break;
       tc_fence_after();
-      uint32_t sr[32];
-      tmem_ld32(tmem + lane_base + b * kAttBlk + 32 * part, sr);
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + kAttColS + b * kAttBlk + 32 * c, sr[c]);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[b]);
+      if (lane == 0) mbar_arrive(&s_empty[b]);  // S_{j+2} may now be written into buffer b
       // Raw scores s' = (float)acc * ks_j (|acc| <= 127^2 * 128 < 2^22, so the bits of
       // acc + 1.5 * 2^23 read as a float, minus 1.5 * 2^23, are (float)acc without the
       // conversion unit); the log2-domain score is s' * cq, cq = qs_i log2(e) / sqrt(128) >= 0,
       // so maxima can be taken on s'. Keys past the end (last block only) are masked.
-      const int key0 = j * kAttBlk + 32 * part;
-      const bool partial = key0 + 32 > S;
-      // the key scales travel with V_j (that stage is released only after P_j V_j)
-      if (!(ok = wait_all(&v_full[st], static_cast<uint32_t>((j / kAttVStages) & 1)))) break;
-      const float* ksb = sKs + st * 128 + 32 * part;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 kv = *reinterpret_cast<const float4*>(ksb + 4 * e4);
-        const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
-        float sc[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * e4 + e;
-          sc[e] = __fmul_rn(__fsub_rn(__uint_as_float(sr[c] + 0x4B400000u), 12582912.0f), kk[e]);
-          if (partial && key0 + c >= S) sc[e] = -INFINITY;
-          sr[c] = __float_as_uint(sc[e]);
-        }
-        mx = att_max3(mx, att_max3(sc[0], sc[1], sc[2]), sc[3]);
+      if (!(ok = wait_all(&v_full[vst], static_cast<uint32_t>((j / kAttVStages) & 1)))) break;
+      const float* ksb = sKs + vst * 128;
+      const int key0 = j * kAttBlk;
+      const bool partial = key0 + kAttBlk > S;
+      const int nvalid = S - key0;  // keys of the block inside the sequence (>= 8)
+      const float mx = partial ? att_scores<true>(sr, ksb, nvalid) : att_scores<false>(sr, ksb, nvalid);
+      if (j > 0) {  // the maximum after block j-1, published by the other set
+        if (!(ok = wait_all(&mx_full[(j - 1) & 1], static_cast<uint32_t>(((j - 1) >> 1) & 1)))) break;
+        adopt(sMx[((j - 1) & 1) * 128 + r]);
       }
-      float* xm = xmax + b * (kAttParts * 128);
-      xm[part * 128 + r] = mx;
-      mbar_arrive(&xchg[b]);
-      if (!(ok = wait_all(&xchg[b], static_cast<uint32_t>((j >> 1) & 1)))) break;
-      mx = att_max3(att_max3(xm[r], xm[128 + r], xm[256 + r]), xm[384 + r], -INFINITY);
       // raise the exponent's maximum when the row maximum grew by more than 2^8 (log2 units)
       const bool need = j == 0 || __fmul_rn(mx - m_used, cq) > 8.0f;
+      const float m_new = need ? mx : m_used;
+      sMx[(j & 1) * 128 + r] = m_new;  // slot j % 2 was last read before the other set published m_{j-1}
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mx_full[j & 1]);
+      if (j >= 2) {  // P buffer b was last read by P_{j-2} V_{j-2}
+        if (!(ok = wait_all(&pv_done[b], static_cast<uint32_t>(((j >> 1) & 1) ^ 1)))) break;
+      }
+      tc_fence_after();
+      // P = 2^(s' cq - m cq) as bf16 pairs (lower key in the low half), 64 keys per store
+      const float nm = -__fmul_rn(m_new, cq);
+      const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(nm, nm);
+      const uint32_t p_cols = tmem + lane_base + kAttColP + b * 64;
+      const float2 bs2 = partial ? att_weights<true>(sr, cq2, nm2, nvalid, p_cols)
+                                 : att_weights<false>(sr, cq2, nm2, nvalid, p_cols);
       if (__ballot_sync(0xFFFFFFFFu, need) != 0u && j > 0) {
-        // O holds P.V of blocks < j with the old maximum: rescale after P_{j-1} V_{j-1} has landed
+        // O holds P.V of blocks < j relative to m_used: rescale it once P_{j-1} V_{j-1} has
+        // landed (P_j V_j waits for this block's P)
         if (!(ok = wait_all(&pv_done[(j - 1) & 1], static_cast<uint32_t>(((j - 1) >> 1) & 1)))) break;
         tc_fence_after();
-        const float f = need ? ex2_approx(__fmul_rn(m_used - mx, cq)) : 1.0f;
-        uint32_t o[32];
-        tmem_ld32(o_cols, o);
-        tmem_ld_wait();
+        const float f = need ? ex2_approx(__fmul_rn(m_used - m_new, cq)) : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + kAttColO + 32 * c, o);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), f));
-        tmem_st32(o_cols, o);
-        tmem_st_wait();
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__fmul_rn(__uint_as_float(o[e]), f));
+          tmem_st32(tmem + lane_base + kAttColO + 32 * c, o);
+        }
         l2 = __fmul2_rn(l2, make_float2(f, f));
       }
-      if (need) m_used = mx;
-      if (j >= 2) {  // P buffer b was last read by P_{j-2} V_{j-2}
-        if (!(ok = wait_all(&pv_done[b], static_cast<uint32_t>(((j - 2) >> 1) & 1)))) break;
-      }
-      // P = 2^(s' cq - m cq) as bf16: this part's 32 keys are chunks 4 (part % 2) .. +3 of row r
-      // of half-tile part / 2 (16-byte chunk c at position c ^ (r % 8) of the 128-byte row)
-      const float nm = -__fmul_rn(m_used, cq);
-      uint8_t* prow = sP + b * kAttPBytes + (part >> 1) * (kAttPBytes / 2) + r * 128;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c0 = 8 * cc + 2 * e;
-          float p0 = ex2_approx(__fmaf_rn(__uint_as_float(sr[c0]), cq, nm));
-          float p1 = ex2_approx(__fmaf_rn(__uint_as_float(sr[c0 + 1]), cq, nm));
-          if (partial) {  // masked keys weigh 0 (also when cq = 0, where -inf * cq is not a number)
-            if (key0 + c0 >= S) p0 = 0.0f;
-            if (key0 + c0 + 1 >= S) p1 = 0.0f;
-          }
-          w[e] = pack_bf16x2(p0, p1);
-          l2 = __fadd2_rn(l2, make_float2(p0, p1));
-        }
-        const int ch = 4 * (part & 1) + cc;
-        *reinterpret_cast<uint4*>(prow + 16 * (ch ^ (r & 7))) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      fence_proxy_async_smem();  // the tensor core reads P through the async proxy
+      m_used = m_new;
+      l2 = __fadd2_rn(l2, bs2);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[b]);
     }
-    if (ok) {
-      const int t = nb - 1;
-      ok = wait_all(&pv_done[t & 1], static_cast<uint32_t>((t >> 1) & 1));
+    // the final maximum is the other set's when it took the last block
+    if (ok && ((nb - 1) & 1) != set) {
+      ok = wait_all(&mx_full[(nb - 1) & 1], static_cast<uint32_t>(((nb - 1) >> 1) & 1));
+      if (ok) adopt(sMx[((nb - 1) & 1) * 128 + r]);
     }
     if (ok) {
-      xsum[part * 128 + r] = __fadd_rn(l2.x, l2.y);
-      mbar_arrive(xsum_bar);
-      ok = wait_all(xsum_bar, 0);
+      sL[set * 128 + r] = __fadd_rn(l2.x, l2.y);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(l_full);
+      ok = wait_all(l_full, 0);
     }
+    if (ok) ok = wait_all(&pv_done[(nb - 1) & 1], static_cast<uint32_t>(((nb - 1) >> 1) & 1));
     if (ok) {
       tc_fence_after();
-      const float lsum = __fadd_rn(__fadd_rn(xsum[r], xsum[128 + r]), __fadd_rn(xsum[256 + r], xsum[384 + r]));
-      const float inv_l = __fdiv_rn(1.0f, lsum);
-      __nv_bfloat16* orow = p.out + int64_t(i) * p.ld_out + h * kAttD + 32 * part;
-      uint32_t o[32];
-      tmem_ld32(o_cols, o);
-      tmem_ld_wait();
-      if (i < S) {
+      const float inv_l = __fdiv_rn(1.0f, __fadd_rn(sL[r], sL[128 + r]));
+      __nv_bfloat16* orow = p.out + int64_t(i) * p.ld_out + h * kAttD + 64 * set;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + kAttColO + 64 * set + 32 * hh, o);
+        tmem_ld_wait();
+        if (i < S) {
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t w[4];
+          for (int g = 0; g < 4; ++g) {
+            uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            w[e] = pack_bf16x2(__fmul_rn(__uint_as_float(o[8 * g + 2 * e]), inv_l),
-                               __fmul_rn(__uint_as_float(o[8 * g + 2 * e + 1]), inv_l));
-          *reinterpret_cast<uint4*>(orow + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack_bf16x2(__fmul_rn(__uint_as_float(o[8 * g + 2 * e]), inv_l),
+                                 __fmul_rn(__uint_as_float(o[8 * g + 2 * e + 1]), inv_l));
+            *reinterpret_cast<uint4*>(orow + 32 * hh + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
     }

@@ -434,11 +434,17 @@ h3q_status h3q_attention_int8(const void* q, const void* k, const void* v, int64
     return H3Q_ERR_CUDA;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
+  static bool regs_ok = false;
   std::call_once(attr_once, [] {
     attr_err = cudaFuncSetAttribute(h3q::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     static_cast<int>(h3q::kAttSmem));
+    cudaFuncAttributes fa{};
+    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, h3q::attn_kernel);
+    // the kernel's register split assumes this many registers per thread at launch
+    regs_ok = attr_err == cudaSuccess && fa.numRegs >= static_cast<int>(h3q::kAttRegsLaunch);
   });
   if (attr_err != cudaSuccess) return H3Q_ERR_CUDA;
+  if (!regs_ok) return H3Q_ERR_UNSUPPORTED;
   h3q::AttParams p{};
   p.S = static_cast<int>(S);
   p.H = static_cast<int>(H);
