@@ -17,11 +17,12 @@
 //            P_j V_j is done);
 //   warp 1   tensor memory (512 columns: two 128-column score buffers, the
 //            128-column output accumulator O and two 64-column P buffers);
-//            one lane issues S_j = Q K_j^T (kind::i8, 128 x 128 x 128) into
-//            score buffer j % 2 as soon as block j-2's scores have been read,
-//            and O += P_j V_j (kind::f16, A = P_j from tensor memory, B = V_j^T
-//            from shared memory, fp32 accumulation) once P_j is written;
-//   warps 2-3 idle;
+//            one lane issues O += P_j V_j (kind::f16, A = P_j from tensor
+//            memory, B = V_j^T from shared memory, fp32 accumulation) once P_j
+//            is written;
+//   warp 3   one lane issues S_j = Q K_j^T (kind::i8, 128 x 128 x 128) into
+//            score buffer j % 2 as soon as block j-2's scores have been read;
+//   warp 2   idle;
 //   warps 4-11 softmax, two sets of four warps, one thread per query row
 //            (tensor-memory lane): set 0 takes the even key blocks, set 1 the
 //            odd ones, so one set's exponentials overlap the other's score
@@ -283,8 +284,9 @@ __global__ void __launch_bounds__(kAttThreads, 1)
   uint64_t* pv_done = bars + 19;  // [P buffer]: P_j V_j has completed
   uint64_t* mx_full = bars + 21;  // [block parity]: the maximum after the block is published
   uint64_t* l_full = bars + 23;   // both sets stored their row sums
-  uint64_t* drain = bars + 24;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 25);
+  uint64_t* drain = bars + 24;     // the P.V issuer's products have completed
+  uint64_t* drain_s = bars + 25;   // the score issuer's products have completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -312,6 +314,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     }
     mbar_init(l_full, 8);
     mbar_init(drain, 1);
+    mbar_init(drain_s, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -359,39 +362,44 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         for (int t = max(0, nv - kAttVStages); t < nv; ++t)
           mbar_wait_bounded(&v_full[t % kAttVStages], static_cast<uint32_t>((t / kAttVStages) & 1), limit, nullptr);
       }
-    } else if (warp == 1) {
+    } else if (warp == 3) {
       if (lane == 0) {
-        // ------------------------------------------------------------ MMA issuer
-        // Order: S_0, S_1, then per block t: S_{t+2} (once S_t has been read), O += P_t V_t.
+        // ------------------------------------------------------------ score issuer
+        // S_j = Q K_j^T into score buffer j % 2 once K_j has landed and S_{j-2} has been
+        // read. A thread of its own, so a score product never queues behind the issue of
+        // a P.V product.
         constexpr uint32_t idesc_s = idesc_i8(kAttBlk, kAttBlk);
-        constexpr uint32_t idesc_o = idesc_bf16(kAttBlk, kAttD);
         bool ok = mbar_wait_bounded(q_full, 0, limit, abort_flag);
         const uint64_t qd = smem_desc_sw128(smem_u32(sQ));
-        auto issue_s = [&](int j) {  // S_j = Q K_j^T into score buffer j % 2
+        for (int j = 0; ok && j < nb; ++j) {
           const int st = j % kAttKStages, b = j & 1;
           if (!mbar_wait_bounded(&k_full[st], static_cast<uint32_t>((j / kAttKStages) & 1), limit, abort_flag) ||
               !mbar_wait_bounded(&s_empty[b], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), limit, abort_flag))
-            return false;
+            break;
           tc_fence_after();
           const uint64_t kd = smem_desc_sw128(smem_u32(sK + st * kAttKBytes));
-  #pragma unroll
+#pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_i8(tmem + kAttColS + b * kAttBlk, qd + 2u * k, kd + 2u * k, idesc_s, k > 0 ? 1u : 0u);
           mma_commit(&s_full[b]);
           mma_commit(&k_empty[st]);
-          return true;
-        };
-        for (int j = 0; ok && j < min(2, nb); ++j) ok = issue_s(j);
-        for (int t = 0; ok && t < nb; ++t) {
-          if (t + 2 < nb && !(ok = issue_s(t + 2))) break;
-          const int bt = t & 1, vst = t % kAttVStages;  // O += P_t V_t
+        }
+        mma_commit(drain_s);
+        mbar_wait_bounded(drain_s, 0, limit, nullptr);
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ------------------------------------------------------------ P.V issuer
+        // O += P_t V_t (kind::f16, A = P_t from tensor memory) once P_t is written and
+        // V_t has landed.
+        constexpr uint32_t idesc_o = idesc_bf16(kAttBlk, kAttD);
+        for (int t = 0; t < nb; ++t) {
+          const int bt = t & 1, vst = t % kAttVStages;
           if (!mbar_wait_bounded(&v_full[vst], static_cast<uint32_t>((t / kAttVStages) & 1), limit, abort_flag) ||
-              !mbar_wait_bounded(&p_full[bt], static_cast<uint32_t>((t >> 1) & 1), limit, abort_flag)) {
-            ok = false;
+              !mbar_wait_bounded(&p_full[bt], static_cast<uint32_t>((t >> 1) & 1), limit, abort_flag))
             break;
-          }
           tc_fence_after();
-  #pragma unroll
+#pragma unroll
           for (int k = 0; k < 8; ++k) {  // 16 keys = 8 P columns = 32 bytes of a V^T row per K step
             const int half = k >> 2;
             const uint64_t vd = smem_desc_sw128(smem_u32(sV + vst * kAttVBytes + half * (kAttVBytes / 2)));
