@@ -166,7 +166,7 @@ h3q_status launch_gemm_fp4(const uint8_t* a, const uint8_t* a_sf, const float* a
   const int sms = sm_count();
   if (sms <= 0) return H3Q_ERR_CUDA;
   const int pairs = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
-  h3q::gemm_fp4_kernel<EPI><<<2 * pairs, h3q::kGemmThreads, h3q::kF4Smem, stream>>>(ta, tb, tsa, tsb, p);
+  h3q::gemm_fp4_kernel<EPI><<<2 * pairs, h3q::kF4Threads, h3q::kF4Smem, stream>>>(ta, tb, tsa, tsb, p);
   return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
 }
 

@@ -218,6 +218,7 @@ constexpr int kF4StageBytes = kF4AStage + kF4BStage + kF4SfaStage + kF4SfbStage;
 constexpr int kF4SfSlots = 4;          // tensor-memory scale-factor slots (48 columns each)
 constexpr int kF4SfCols = 48;          // per slot: SFA 16 columns, SFB 32 columns
 constexpr size_t kF4Smem = size_t(kF4Stages) * kF4StageBytes + 1024 + 256 + 2 * kBN * 4;
+constexpr int kF4Threads = kGemmThreads + 32;  // producer, MMA, 8 epilogue warps, scale copier
 
 struct Fp4Params {
   int M, N, K;              // N: output columns (SwiGLU: F); K in elements
@@ -242,7 +243,7 @@ __device__ __forceinline__ void fp4_tile_coords(int tile, const Fp4Params& p, in
 
 // EPI: kEpiS32 = raw fp32 accumulators (test hook), kEpiBF16, kEpiSwiGLU.
 template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kF4Threads, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                     const Fp4Params p) {
@@ -257,7 +258,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + kF4Stages;
   uint64_t* tempty = tfull + 1;
   uint64_t* drain = tempty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sf_full = drain + 1;              // [slot] (leader): a stage's scales are in tensor memory
+  uint64_t* sf_empty = sf_full + kF4SfSlots;  // [slot] (leader): the MMAs that read the slot are done
+  uint64_t* drain_cp = sf_empty + kF4SfSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_cp + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* col_bias = reinterpret_cast<float*>(smem + kF4Stages * kF4StageBytes + 256);  // [2][kBN]
 
@@ -276,6 +280,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     mbar_init(tfull, 1);
     mbar_init(tempty, 16);
     mbar_init(drain, 1);
+    for (int s = 0; s < kF4SfSlots; ++s) {
+      mbar_init(&sf_full[s], 1);
+      mbar_init(&sf_empty[s], 1);
+    }
+    mbar_init(drain_cp, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -345,6 +354,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_phase = 0;
+      long nk = 0;  // stages consumed, across tiles: scale slot nk % kF4SfSlots
       bool ok = true;
       for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
         if (!mbar_wait_bounded_cluster(tempty, acc_phase ^ 1u, limit, abort_flag)) break;
@@ -354,16 +364,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t sf_col = tmem + static_cast<uint32_t>(kBN + (stage % kF4SfSlots) * kF4SfCols);
-          const uint32_t sfa_base = smem_u32(sSFA + stage * kF4SfaStage);
-          const uint32_t sfb_base = smem_u32(sSFB + stage * kF4SfbStage);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_cp_32x128b_x4_pair(sf_col + 4 * j, smem_desc_sf_atom(sfa_base + 512 * j));
-            tmem_cp_32x128b_x4_pair(sf_col + 16 + 8 * j, smem_desc_sf_atom(sfb_base + 512 * j));
-            tmem_cp_32x128b_x4_pair(sf_col + 16 + 8 * j + 4, smem_desc_sf_atom(sfb_base + 2048 + 512 * j));
+          const int slot = static_cast<int>(nk % kF4SfSlots);
+          if (!mbar_wait_bounded(&sf_full[slot], static_cast<uint32_t>((nk / kF4SfSlots) & 1), limit, abort_flag)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t sf_col = tmem + static_cast<uint32_t>(kBN + slot * kF4SfCols);
           const uint64_t ad = smem_desc_sw128(smem_u32(sA + stage * kF4AStage));
           const uint64_t bd = smem_desc_sw128(smem_u32(sB + stage * kF4BStage));
 #pragma unroll
@@ -372,6 +379,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                          (kb | k) != 0 ? 1u : 0u);
           mma_commit_pair(cluster_map(&empty[stage], 0));
           mma_commit_pair(cluster_map(&empty[stage], 1));
+          mma_commit_pair(cluster_map(&sf_empty[slot], 0));
+          ++nk;
           if (++stage == kF4Stages) {
             stage = 0;
             phase ^= 1u;
@@ -384,6 +393,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       mma_commit_pair(cluster_map(drain, 0));
       mbar_wait_bounded(drain, 0, limit, nullptr);
+    }
+  } else if (warp == kF4Threads / 32 - 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------------ scale copier (leader only)
+      // Copies each stage's block scales into tensor-memory slot n % kF4SfSlots (12
+      // tcgen05.cp per stage, into both CTAs) once the stage has landed and the MMAs
+      // that last read the slot are done, and signals the MMA issuer through sf_full.
+      // A thread of its own: the copies no longer queue in the MMA issuer's stream.
+      int stage = 0;
+      uint32_t phase = 0;
+      long n = 0;
+      for (int tile = pair; tile < p.num_tiles; tile += npairs) {
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          const int slot = static_cast<int>(n % kF4SfSlots);
+          if (!mbar_wait_bounded(&full[stage], phase, limit, abort_flag) ||
+              !mbar_wait_bounded(&sf_empty[slot], static_cast<uint32_t>(((n / kF4SfSlots) & 1) ^ 1), limit,
+                                 abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sf_col = tmem + static_cast<uint32_t>(kBN + slot * kF4SfCols);
+          const uint32_t sfa_base = smem_u32(sSFA + stage * kF4SfaStage);
+          const uint32_t sfb_base = smem_u32(sSFB + stage * kF4SfbStage);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tmem_cp_32x128b_x4_pair(sf_col + 4 * j, smem_desc_sf_atom(sfa_base + 512 * j));
+            tmem_cp_32x128b_x4_pair(sf_col + 16 + 8 * j, smem_desc_sf_atom(sfb_base + 512 * j));
+            tmem_cp_32x128b_x4_pair(sf_col + 16 + 8 * j + 4, smem_desc_sf_atom(sfb_base + 2048 + 512 * j));
+          }
+          mma_commit_pair(cluster_map(&sf_full[slot], 0));
+          ++n;
+          if (++stage == kF4Stages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      mma_commit_pair(cluster_map(drain_cp, 0));
+      mbar_wait_bounded(drain_cp, 0, limit, nullptr);
     }
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
