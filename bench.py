@@ -892,7 +892,8 @@ def run_attention(args):
             "context_library_bf16_sdpa": {"ms": sdpa_ms, "backend": sdpa_backend,
                                           "note": "library bf16 attention on the same tensors; context, not a target"},
             "roofline": {"bound": "tensor", "kernel": "attn_kernel (+ attn_prep_kernel)", "achieved": achieved,
-                         "peak": mixed, "unit": "TFLOP/s", "frac": achieved / mixed, "traffic": None,
+                         "peak": mixed, "unit": "TFLOP/s", "frac": achieved / mixed,
+                         "traffic": traffic_from_profile("attn_kernel_attention"),
                          "peak_source": f"{peak_src}: half the flops at the int8 rate (2 x bf16 burst) and half at "
                                         f"the bf16 burst rate {peaks['bf16_tflops']} TFLOP/s"},
             "gpu_launches": 2 * steps,
