@@ -67,7 +67,8 @@ constexpr int kAttKsBytes = 128 * 4;       // the key block's scales
 constexpr uint32_t kAttColS = 0;    // score buffers b at b * 128 (int32)
 constexpr uint32_t kAttColO = 256;  // output accumulator (fp32)
 constexpr uint32_t kAttColP = 384;  // P buffers b at 384 + b * 64 (bf16 pairs)
-constexpr size_t kAttSmem = size_t(kAttQBytes) + kAttKStages * kAttKBytes +
+constexpr int kAttBiasBytes = 2 * 128 * 128;  // the bias product's two bf16 operands (128 x 64, swizzled)
+constexpr size_t kAttSmem = size_t(kAttBiasBytes) + kAttQBytes + kAttKStages * kAttKBytes +
                             kAttVStages * (size_t(kAttVBytes) + kAttKsBytes) + 2 * 128 * 4 /*maxima*/ +
                             2 * 128 * 4 /*row sums*/ + 1024 + 256;
 
@@ -108,6 +109,17 @@ __device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32, one CTA.
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // kind::f16 with bf16 A and B, fp32 accumulator, K-major operands.
 __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N) {
   return (1u << 4)             // D format: f32
@@ -140,9 +152,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 // Scales a block's raw scores in place, s'_k = (float)acc_k * ks_k, and returns
-// their maximum. |acc| <= 127^2 * 128 < 2^22, so the bits of acc + 1.5 * 2^23
-// read as a float, minus 1.5 * 2^23, are (float)acc exactly, without the
-// conversion unit. With kMasked, keys k >= nvalid (past the end of the
+// their maximum. The accumulators start from the fp32 bits of 1.5 * 2^23 (written
+// by a bf16 product before the int8 ones), so they hold 0x4B400000 + acc; with
+// |acc| <= 127^2 * 128 < 2^22 those bits read as a float are 1.5 * 2^23 + acc
+// exactly, and one subtraction gives (float)acc, without the conversion unit. With kMasked, keys k >= nvalid (past the end of the
 // sequence) get s' = -inf; the two forms are separate so the unmasked one,
 // used for every block but the last, carries no per-key predicates.
 template <bool kMasked>
@@ -155,9 +168,8 @@ __device__ __forceinline__ float att_scores(uint32_t (&sr)[4][32], const float* 
     for (int e4 = 0; e4 < 8; ++e4) {
       const int k0 = 4 * e4;
       const float4 kv = *reinterpret_cast<const float4*>(ksb + 32 * c + k0);
-      float2 x01 = make_float2(__uint_as_float(sr[c][k0] + 0x4B400000u), __uint_as_float(sr[c][k0 + 1] + 0x4B400000u));
-      float2 x23 =
-          make_float2(__uint_as_float(sr[c][k0 + 2] + 0x4B400000u), __uint_as_float(sr[c][k0 + 3] + 0x4B400000u));
+      float2 x01 = make_float2(__uint_as_float(sr[c][k0]), __uint_as_float(sr[c][k0 + 1]));
+      float2 x23 = make_float2(__uint_as_float(sr[c][k0 + 2]), __uint_as_float(sr[c][k0 + 3]));
       x01 = __fmul2_rn(__fadd2_rn(x01, magic2), make_float2(kv.x, kv.y));
       x23 = __fmul2_rn(__fadd2_rn(x23, magic2), make_float2(kv.z, kv.w));
       float sc[4] = {x01.x, x01.y, x23.x, x23.y};
@@ -266,7 +278,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 const __grid_constant__ CUtensorMap tmV, const AttParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
+  uint8_t* sBias = smem;                           // [2][128 rows x 128 B]: A = e_0, B = 1.5 * 2^23 e_0
+  uint8_t* sQ = sBias + kAttBiasBytes;
   uint8_t* sK = sQ + kAttQBytes;                   // [K stage][128 keys x 128 B]
   uint8_t* sV = sK + kAttKStages * kAttKBytes;     // [V stage][2 boxes: 128 d rows x 64 keys (128 B)]
   float* sKs = reinterpret_cast<float*>(sV + kAttVStages * kAttVBytes);  // [V stage][128] key scales
@@ -295,6 +308,17 @@ __global__ void __launch_bounds__(kAttThreads, 1)
   const int nb = (S + kAttBlk - 1) / kAttBlk;
   const uint64_t limit = p.wait_limit_ns;
 
+  // The bias product: A = e_0 (bf16 1.0 in column 0 of every row), B = 1.5 * 2^23 e_0, so
+  // A B^T writes the fp32 value 1.5 * 2^23 (bits 0x4B400000) into every score element; the
+  // int8 products then accumulate onto those bits as int32 (128-byte swizzle: element 0 of
+  // row m sits in 16-byte chunk m % 8).
+  for (int e = threadIdx.x; e < kAttBiasBytes / 16; e += blockDim.x) {
+    const int op = e / 1024, row = (e >> 3) & 127, chunk = e & 7;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (chunk == (row & 7)) v.x = op == 0 ? 0x3F80u : 0x4B40u;
+    reinterpret_cast<uint4*>(sBias)[e] = v;
+  }
+  fence_proxy_async_smem();  // the tensor core reads them through the async proxy
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int st = 0; st < kAttKStages; ++st) {
@@ -369,6 +393,9 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         // read. A thread of its own, so a score product never queues behind the issue of
         // a P.V product.
         constexpr uint32_t idesc_s = idesc_i8(kAttBlk, kAttBlk);
+        constexpr uint32_t idesc_bias = idesc_bf16(kAttBlk, kAttBlk);
+        const uint64_t bias_a = smem_desc_sw128(smem_u32(sBias));
+        const uint64_t bias_b = smem_desc_sw128(smem_u32(sBias + kAttBiasBytes / 2));
         bool ok = mbar_wait_bounded(q_full, 0, limit, abort_flag);
         const uint64_t qd = smem_desc_sw128(smem_u32(sQ));
         for (int j = 0; ok && j < nb; ++j) {
@@ -378,9 +405,11 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             break;
           tc_fence_after();
           const uint64_t kd = smem_desc_sw128(smem_u32(sK + st * kAttKBytes));
+          // bias 1.5 * 2^23 (fp32 bits 0x4B400000), then the int8 products on top of it
+          mma_bf16_ss(tmem + kAttColS + b * kAttBlk, bias_a, bias_b, idesc_bias, 0u);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_i8(tmem + kAttColS + b * kAttBlk, qd + 2u * k, kd + 2u * k, idesc_s, k > 0 ? 1u : 0u);
+            mma_i8(tmem + kAttColS + b * kAttBlk, qd + 2u * k, kd + 2u * k, idesc_s, 1u);
           mma_commit(&s_full[b]);
           mma_commit(&k_empty[st]);
         }
