@@ -149,7 +149,7 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         from datetime import datetime
-        rows = []
+        samples = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 10:
@@ -158,9 +158,13 @@ class ClockSampler:
                 ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
             except ValueError:
                 continue
-            if t0 is not None and not (t0 <= ts <= t1):
-                continue
-            rows.append(parts[1:])
+            samples.append((ts, parts[1:]))
+        window = "timed region"
+        rows = [r for ts, r in samples if t0 is None or t0 <= ts <= t1]
+        if not rows and t0 is not None:
+            # a timed region shorter than the sampling interval: the samples just around it
+            rows = [r for ts, r in samples if t0 - 0.15 <= ts <= t1 + 0.15]
+            window = "nearest samples (timed region shorter than the 100 ms sampling interval)"
         if not rows:
             return None
 
@@ -176,7 +180,7 @@ class ClockSampler:
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
         load = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
         return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
-                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(rows)}
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(rows), "window": window}
 
 
 # ----------------------------------------------------------------------------- oracle rate
