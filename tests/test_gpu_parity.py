@@ -49,7 +49,10 @@ def assert_bf16_close(got, want, where):
 
 # ---------------------------------------------------------------- rotate + quantize
 @pytest.mark.parametrize("M,K", [(1, 256), (7, 512), (64, 512), (129, 768), (300, 5376), (33, 14336),
-                                 (5, 16384), (130, 1280), (17, 256)])
+                                 (5, 16384), (130, 1280), (17, 256),
+                                 # the split-role kernel (groups per row a multiple of 28): more rows than
+                                 # SMs, so blocks cycle their ring and both row buffers; one group per role
+                                 (300, 14336), (20, 7168)])
 def test_rotate_quant_bitexact(h3q, cuda_device, M, K):
     bits, to_dev = _u(cuda_device)
     f = synth.column_factors(K, synth.outlier_columns(0, 4, K, max(1, K // 100)), 50.0)
