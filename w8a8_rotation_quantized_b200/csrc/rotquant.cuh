@@ -369,12 +369,13 @@ RqShape rotquant_plan(int K, int dev, int* blocks_per_sm) {
   RqShape best{0, 0, 0, 0, false};
   int best_occ = 0;
   double best_score = -1.0;
-  // Shapes measured fastest on B200 for the H3 widths (bf16 rows, M = 16384):
-  // K = 5376: 2 groups per slot, 3 rows per item, 16 consumer warps, 4 stages
-  // (2.92 TB/s, against 2.57 for the best one-group shape); K = 14336: one group
-  // per slot, 28 consumer warps, 4 stages (2.95 TB/s).
-  if (sizeof(T) == 2 && (K == 5376 || K == 14336)) {
-    const RqShape pick = K == 5376 ? RqShape{2, 16, 3, 4, false} : RqShape{1, 28, 1, 4, false};
+  // Shapes measured fastest on B200 (bf16 rows, M = 16384): K = 5376: 2 groups per
+  // slot, 3 rows per item, 16 consumer warps, 4 stages (2.92 TB/s, against 2.57 for
+  // the best one-group shape); rows of 32 to 62 groups: one group per slot, one row
+  // per item, ceil(G / 2) consumer warps, 4 stages (K = 14336: 28 warps, 2.95 TB/s;
+  // K = 10752: 21 warps, 2.56 TB/s against 2.05 for the planner's choice).
+  if (sizeof(T) == 2 && (K == 5376 || (G >= 32 && G <= 62))) {
+    const RqShape pick = K == 5376 ? RqShape{2, 16, 3, 4, false} : RqShape{1, (G + 1) / 2, 1, 4, false};
     const uint32_t stage_bytes = static_cast<uint32_t>(int64_t(pick.rows) * K * int64_t(sizeof(T)));
     const int occ = rotquant_occupancy<T>(pick.gps, pick.small, 32 * (pick.warps + 1),
                                           rotquant_smem_bytes(pick.stages, stage_bytes, pick.warps), dev);
