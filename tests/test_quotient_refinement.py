@@ -18,3 +18,18 @@ def test_refined_quotient_equals_ieee_division(tmp_path):
     bad, cases = map(int, out.stdout.split())
     assert cases == 40_000_000
     assert bad == 0, out.stderr
+
+
+def test_division_by_127_in_one_correction_step(tmp_path):
+    """The per-row scale s = max / 127 is formed as RN(max * RN(1/127)) plus one FMA
+    correction; that equals the IEEE quotient for every positive finite float (a full
+    sweep, about a minute, with H3Q_FULL_DIV127_SWEEP=1; by default every 61st bit
+    pattern, which still covers every exponent and mantissa residue class mod 61)."""
+    exe = tmp_path / "div127_check"
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-o", str(exe),
+                           os.path.join(HERE, "csrc", "div127_check.c"), "-lm"])
+    stride = "1" if os.environ.get("H3Q_FULL_DIV127_SWEEP") == "1" else "61"
+    out = subprocess.run([str(exe), stride], capture_output=True, text=True, check=True)
+    checked, wrong = map(int, out.stdout.split())
+    assert checked >= 0x7F800000 // int(stride) - 1
+    assert wrong == 0, out.stderr

@@ -145,6 +145,15 @@ struct RowQuot {
   float f, sf, rs;
 };
 
+// s = RN(a / 127) for a >= 0: RN(a RN(1/127)) and one FMA correction step, which
+// returns the IEEE quotient for every non-negative float (an exhaustive host check
+// over all 2^31 - 2^23 finite positive patterns), in three dependent operations.
+__device__ __forceinline__ float div127(float a) {
+  constexpr float c = 1.0f / 127.0f;
+  const float q0 = __fmul_rn(a, c);
+  return __fmaf_rn(__fmaf_rn(-q0, 127.0f, a), c, q0);
+}
+
 __device__ __forceinline__ RowQuot row_quotient(float s16) {
   RowQuot r;
   r.f = s16 < 0x1p-100f ? 0x1p64f : 1.0f;
@@ -155,13 +164,16 @@ __device__ __forceinline__ RowQuot row_quotient(float s16) {
 
 // int8 codes rne(y16 / s16) of this lane's column hl, written as bytes into the
 // group's 256-byte code buffer at element positions 16 r + hl and 16 (r + 8) + hl.
+// kRescaled: the row's f is 2^64 (scale below 2^-100); otherwise f = 1 and the exact
+// rescaling is skipped.
+template <bool kRescaled>
 __device__ __forceinline__ void quantize_column(const float2 (&p)[8], const RowQuot& rq, int hl,
                                                 uint8_t* codes) {
   const float2 magic = make_float2(12582912.0f, 12582912.0f);
   const float2 f2 = make_float2(rq.f, rq.f), r2 = make_float2(rq.rs, rq.rs), ns2 = make_float2(-rq.sf, -rq.sf);
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
-    const float2 y = __fmul2_rn(p[r], f2);  // exact
+    const float2 y = kRescaled ? __fmul2_rn(p[r], f2) : p[r];  // exact
     float2 q = __fmul2_rn(y, r2);
     float2 e = __ffma2_rn(q, ns2, y);
     q = __ffma2_rn(e, r2, q);
@@ -310,9 +322,13 @@ __global__ void __launch_bounds__(SMALL ? 512 : (GPS == 1 ? 1024 : 544), SMALL ?
     for (int t = 0; t < GPS; ++t) {
       const int64_t row = row0 + rr[t];
       const float am = __uint_as_float(row_amax[buf * kRqMaxRows + rr[t]]);
-      const float s16 = __fdiv_rn(am, 127.0f);
+      const float s16 = div127(am);
       if (hl == 0 && gg[t] == 0 && act[t] && row < a.M) a.s_out[row] = __fmul_rn(s16, 0.0625f);
-      quantize_column(p[t], row_quotient(s16), hl, codes_buf);
+      const RowQuot rq = row_quotient(s16);
+      if (rq.f == 1.0f)
+        quantize_column<false>(p[t], rq, hl, codes_buf);
+      else
+        quantize_column<true>(p[t], rq, hl, codes_buf);
       __syncwarp();
       const uint4 out = *reinterpret_cast<const uint4*>(codes_buf + 16 * hl);  // elements 16 hl .. 16 hl + 15
       __syncwarp();  // before the buffer is reused
