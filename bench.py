@@ -779,6 +779,40 @@ def run_nvfp4(args):
     return 0
 
 
+def oracle_rotquant_rate(K, target_s):
+    """The oracle's rotate+quantize of bf16 activation rows of width K on a bounded sample
+    of rows, on all host cores and on one core; GB/s of 2 B read + 1 B written per element
+    + 4 B per row, as the GPU kernel's figure."""
+    import numpy as np
+
+    import oracle
+    import synth
+    ids = synth.tensor_ids()
+    factors = synth.column_factors(K, synth.outlier_columns(0, ids["outlier"], K, int(round(0.01 * K))), 50.0)
+    x = synth.activation_host(0, ids["x"], np.arange(4096), K, factors)
+    cores = oracle.num_threads()
+
+    def rate(threads, budget):
+        oracle.set_num_threads(threads)
+        rows = 16
+        while True:
+            t0 = time.perf_counter()
+            oracle.rotate_quant_bf16(x[:rows])
+            dt = time.perf_counter() - t0
+            if dt >= budget or rows >= x.shape[0]:
+                break
+            rows = min(x.shape[0], max(rows * 2, int(rows * budget / max(dt, 1e-4) * 1.1)))
+        return (3.0 * rows * K + 4.0 * rows) / dt / 1e9, rows, dt
+    try:
+        all_gbs, all_rows, all_dt = rate(cores, target_s)
+        one_gbs, one_rows, one_dt = rate(1, target_s)
+    finally:
+        oracle.set_num_threads(cores)
+    return {"unit": "GB/s", "kind": "oracle", "K": K,
+            "all_cores": {"value": all_gbs, "cores": cores, "sample": f"{all_rows} rows, {all_dt:.1f} s"},
+            "one_core": {"value": one_gbs, "cores": 1, "sample": f"{one_rows} rows, {one_dt:.1f} s"}}
+
+
 def oracle_nvfp4_rate(target_s):
     """The oracle's NVFP4 layer on a bounded sample of rows of the QKV projection
     (full weight); GEMM flops per second."""
@@ -1216,6 +1250,11 @@ def run_gpu(args):
                                                    args.cpu_seconds)
             except Exception as exc:  # the line still prints; the reason is kept
                 line["cpu_baseline"] = {"value": None, "error": repr(exc)}
+            if spec.name in ("ffn", "qkv", "out"):  # the rotate+quantize oracle alone, all cores and one
+                try:
+                    line["cpu_baseline_rotquant"] = oracle_rotquant_rate(K, min(2.0, args.cpu_seconds))
+                except Exception as exc:
+                    line["cpu_baseline_rotquant"] = {"value": None, "error": repr(exc)}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -54,6 +54,7 @@ def _load():
             "orc_linear": (I64, [P, I64, I64, P, P, I64, P, ctypes.c_int, P, P, P, P, P]),
             "orc_ffn": (I64, [P, I64, I64, P, P, P, I64, P, P, P, P, P, P, P]),
             "orc_num_threads": (ctypes.c_int, []),
+            "orc_set_num_threads": (None, [ctypes.c_int]),
             "orc_lora_merge": (None, [P, P, I64, I64, P, P, I64, F]),
             "orc_f32_to_bf16": (ctypes.c_uint16, [F]),
             "orc_bf16_to_f32": (F, [ctypes.c_uint16]),
@@ -84,6 +85,11 @@ def _c(a, dtype):
 
 def num_threads() -> int:
     return int(_load().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Thread count of the oracle's parallel loops from now on (for timing on one core)."""
+    _load().orc_set_num_threads(int(n))
 
 
 def f32_to_bf16(v: float) -> int:

@@ -552,4 +552,13 @@ int orc_num_threads(void) {
 #endif
 }
 
+// Thread count of the following parallel loops (timing on one core); n <= 0 is ignored.
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 }  // extern "C"
