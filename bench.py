@@ -45,6 +45,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -132,10 +133,10 @@ class ClockSampler:
 
     def start(self):
         try:
-            self.path = f"/tmp/h3q_clocks_{os.getpid()}.csv"
+            fd, self.path = tempfile.mkstemp(prefix="h3q_clocks_", suffix=".csv")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                                         stdout=os.fdopen(fd, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -150,7 +151,13 @@ class ClockSampler:
             self.proc.kill()
         from datetime import datetime
         samples = []
-        for line in open(self.path):
+        with open(self.path) as f:
+            lines = f.readlines()
+        try:
+            os.unlink(self.path)
+        except OSError:
+            pass
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 10:
                 continue

@@ -57,9 +57,9 @@ enum { H3Q_EPI_NONE = 0, H3Q_EPI_SWIGLU = 1 };
 #define H3Q_MAX_K 16384
 
 /*
- * Rotate + per-token quantize (h3-rs README, "What makes it fast": the ConvRot
- * Hadamard rotation is done warp-level inside the quantizer, activations are
- * quantized per row).
+ * Rotate + per-token quantize (h3-rs README, "What makes it fast": the quantizer
+ * itself applies the ConvRot Hadamard rotation, at warp level, and each row of
+ * activations gets its own scale).
  *   x_bf16 [M, K] bf16 in; xq [M, K] int8 out (rotated codes); sx [M] fp32 out.
  *   K % 256 == 0, 256 <= K <= H3Q_MAX_K; M >= 1 (M == 0 is a no-op).
  */
@@ -76,8 +76,8 @@ h3q_status h3q_prepare_weight(const float* w, int64_t N, int64_t K, int8_t* wq, 
                               cudaStream_t stream);
 
 /*
- * W8A8 linear with fused epilogue (h3-rs README, "What makes it fast": the fused
- * int8 GEMM writes bf16 directly; fc1's SwiGLU fuses into its epilogue).
+ * W8A8 linear with fused epilogue (h3-rs README, "What makes it fast": the int8
+ * GEMM produces bf16 itself, and for fc1 the SwiGLU runs inside its epilogue).
  *   acc[m][n] = sum_k xq[m][k] * wq[n][k] (exact int32);
  *   v = ((float)acc * sx[m]) * sw[n] (+ bias[n]), fp32, no fused multiply-add.
  *   epilogue H3Q_EPI_NONE:   y [M, N] bf16 = bf16_rne(v).
@@ -143,8 +143,9 @@ h3q_status h3q_ffn_static_scratch(const void* x_bf16, int64_t M, int64_t K,
 
 /*
  * LoRA merge into stored int8 weights (h3-rs README, "Speed", "What makes it
- * fast": LoRAs are merged into the int8 weights at load by dequantizing,
- * adding and requantizing, so they cost nothing per step). The codes are in the
+ * fast": a LoRA is folded into the int8 weights once, when the model loads, by
+ * dequantizing, adding and requantizing, so inference steps pay nothing for
+ * it). The codes are in the
  * rotated basis, so the delta is rotated the same way:
  *   A_rot = A blockdiag(H/16) (the rotation of h3q_prepare_weight, fp32);
  *   d[n][k] = fma chain over j = 0..r-1 ascending, from 0, of B[n][j] A_rot[j][k];

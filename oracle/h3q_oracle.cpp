@@ -301,8 +301,8 @@ int64_t orc_ffn(const uint16_t* x, int64_t M, int64_t K, const int8_t* w_gu, con
 
 // ---------------------------------------------------------------------------
 // LoRA merge into stored rotated int8 weights (h3-rs README, "What makes it
-// fast": LoRAs are merged into the int8 weights at load: dequantize, add,
-// requantize). The stored codes are in the rotated basis, so the low-rank delta
+// fast": a LoRA is folded into the int8 weights once, at model load, by
+// dequantizing, adding and requantizing). The stored codes are in the rotated basis, so the low-rank delta
 // alpha * B A (B [N, r], A [r, K] in the model's basis) is rotated along K the
 // same way: A_rot = A blockdiag(H/16), delta = alpha * B A_rot. Per element, in
 // fp32 and in this order: d = sum over j ascending of B[n][j] * A_rot[j][k] as a

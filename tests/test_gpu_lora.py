@@ -1,8 +1,8 @@
 """LoRA merge into rotated int8 weights on the GPU, element by element against
 the oracle: codes bit-exact, scales bit-exact.
 
-The merge (h3-rs README, "Speed", "What makes it fast": LoRAs are merged into
-the int8 weights at load by dequantizing, adding and requantizing) rotates A
+The merge (h3-rs README, "Speed", "What makes it fast": a LoRA is folded into
+the int8 weights once, at model load, by dequantizing, adding and requantizing) rotates A
 along K, forms alpha * B A_rot in fp32 in a fixed order and requantizes each
 row; both sides take every rounding in the same order, so nothing differs.
 Cases cover ragged row blocks, every cluster width the launch picks (one CTA

@@ -50,9 +50,8 @@ def assert_bf16_close(got, want, where):
 # ---------------------------------------------------------------- rotate + quantize
 @pytest.mark.parametrize("M,K", [(1, 256), (7, 512), (64, 512), (129, 768), (300, 5376), (33, 14336),
                                  (5, 16384), (130, 1280), (17, 256),
-                                 # the split-role kernel (groups per row a multiple of 28): more rows than
-                                 # SMs, so blocks cycle their ring and both row buffers; one group per role
-                                 (300, 14336), (20, 7168)])
+                                 # more rows than SMs, so blocks cycle their ring and the row buffers
+                                 (300, 14336), (20, 7168), (1000, 5376), (601, 10752)])
 def test_rotate_quant_bitexact(h3q, cuda_device, M, K):
     bits, to_dev = _u(cuda_device)
     f = synth.column_factors(K, synth.outlier_columns(0, 4, K, max(1, K // 100)), 50.0)
@@ -74,7 +73,9 @@ def test_rotate_quant_bitexact(h3q, cuda_device, M, K):
     assert np.array_equal(xq.cpu().numpy(), oq)
 
 
-@pytest.mark.parametrize("N,K", [(256, 512), (264, 5376), (8, 14336), (3, 256)])
+# fp32 rows longer than 8192 are copied as two boxes per row (a box holds at most
+# 256 units of 128 bytes); K = 8448 splits a group across the two boxes.
+@pytest.mark.parametrize("N,K", [(256, 512), (264, 5376), (8, 14336), (3, 256), (5, 8448), (3, 16384)])
 def test_prepare_weight_bitexact(h3q, cuda_device, N, K):
     w_h = synth.weight_host(0, 2, np.arange(N), K)
     w_h[N // 2, 7] = 3.0  # an outlier weight
@@ -86,6 +87,40 @@ def test_prepare_weight_bitexact(h3q, cuda_device, N, K):
     oq, os_ = oracle.prepare_weight(w_h)
     assert np.array_equal(sw.cpu().numpy().view(np.uint32), os_.view(np.uint32))
     assert np.array_equal(wq.cpu().numpy(), oq)
+
+
+def test_prepare_weight_half_integer_quotients(h3q, cuda_device):
+    """Weight rows a e0 + b e1 with a + b = 254 and a - b = m odd: the first group
+    rotates to values (a + b)/16 and (a - b)/16, so s = 0.125 and the smaller values
+    give the quotient m/2, exactly half-integer; with b moved by 1 or 4 ulps the
+    quotients sit a few ulps from the half-integers. There the kernel's candidate
+    code fails its residual check and the exactly rounded quotient decides."""
+    K = 512
+    rows = []
+    for m in range(1, 254, 2):
+        a = np.float32((254 + m) / 2)
+        for db in (0, 1, -1, 4, -4):
+            b = np.float32((254 - m) / 2)
+            for _ in range(abs(db)):
+                b = np.nextafter(b, np.float32(np.inf if db > 0 else -np.inf), dtype=np.float32)
+            w = np.zeros(K, dtype=np.float32)
+            w[0], w[1] = a, b
+            w[300] = np.float32(0.001 * m)  # second group: ordinary values
+            rows.append(w)
+    w_h = np.stack(rows)
+    N = w_h.shape[0]
+    w = torch.from_numpy(w_h).to(cuda_device)
+    wq = torch.empty((N, K), dtype=torch.int8, device=cuda_device)
+    sw = torch.empty(N, dtype=torch.float32, device=cuda_device)
+    h3q.h3q_prepare_weight(w, wq, sw)
+    torch.cuda.synchronize()
+    oq, os_ = oracle.prepare_weight(w_h)
+    assert np.array_equal(sw.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    got = wq.cpu().numpy()
+    assert np.array_equal(got, oq)
+    # the exact ties round half to even: m/2 -> the even neighbour
+    ties = got[0::5, :256]
+    assert set(np.unique(np.abs(ties[:, 1::2]) % 2)) <= {0}
 
 
 # ---------------------------------------------------------------- int8 GEMM

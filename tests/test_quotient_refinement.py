@@ -33,3 +33,19 @@ def test_division_by_127_in_one_correction_step(tmp_path):
     checked, wrong = map(int, out.stdout.split())
     assert checked >= 0x7F800000 // int(stride) - 1
     assert wrong == 0, out.stderr
+
+
+def test_candidate_code_with_residual_check_equals_rounded_ieee_quotient(tmp_path):
+    """The kernel's code decision: candidate rne(y rs) accepted when its residual
+    |y - n s| is at most RN(s (1/2 - 2^-16)), else the refined quotient rounded half
+    to even. Compared with rintf(y / s) on 40 M cases, a third of them exact
+    half-integer quotients and a third within four ulps of one; the exact ties must
+    all take the fallback."""
+    exe = tmp_path / "code_check"
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-o", str(exe),
+                           os.path.join(HERE, "csrc", "code_check.c"), "-lm"])
+    out = subprocess.run([str(exe), "2000", "20000"], capture_output=True, text=True, check=True)
+    bad, cases, fallbacks = map(int, out.stdout.split())
+    assert cases == 40_000_000
+    assert bad == 0, out.stderr
+    assert fallbacks >= cases // 3

@@ -184,6 +184,39 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t co
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Rows of K elements (bf16 or fp32) seen as [rows][K * size / 128][128 bytes]
+// for the rotate+quantize stages: boxes of `units` 128-byte units x `box_rows`
+// rows, 128-byte swizzle; rows past the end read as zeros.
+bool make_tmap_rows(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int elem_bytes, int units,
+                    int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(128 / elem_bytes),
+                              static_cast<cuuint64_t>(K * elem_bytes / 128), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(K * elem_bytes)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(units),
+                             static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T>
+h3q_status run_rotquant(const T* x, int64_t rows, int64_t K, int8_t* q, float* s, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return H3Q_ERR_CUDA;
+  int occ = 0;
+  const h3q::RqShape sh = h3q::rotquant_plan<T>(static_cast<int>(K), dev, &occ);
+  if (sh.gps == 0 || occ < 1) return H3Q_ERR_CUDA;
+  const h3q::RqArgs a = h3q::rotquant_args<T>(sh, rows, K, q, s, g_wait_limit_ns.load());
+  CUtensorMap map;
+  if (!make_tmap_rows(&map, x, rows, K, static_cast<int>(sizeof(T)), a.units_per_copy, sh.rows))
+    return H3Q_ERR_CUDA;
+  return h3q::launch_rotquant<T>(map, sh, occ, a, stream) == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+}
+
 bool valid_k(int64_t K) { return K >= 256 && K % 256 == 0; }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -247,9 +280,7 @@ h3q_status h3q_rotate_quant(const void* x_bf16, int64_t M, int64_t K, int8_t* xq
   if (M == 0) return H3Q_OK;
   if (!x_bf16 || !xq || !sx || !aligned16(x_bf16) || !aligned16(xq) || !aligned16(sx)) return H3Q_ERR_INVALID_ARG;
   if (K > H3Q_MAX_K || M > INT32_MAX) return H3Q_ERR_UNSUPPORTED;
-  const cudaError_t e = h3q::launch_rotquant(static_cast<const __nv_bfloat16*>(x_bf16), M, K, xq, sx,
-                                             g_wait_limit_ns.load(), stream);
-  return e == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+  return run_rotquant(static_cast<const __nv_bfloat16*>(x_bf16), M, K, xq, sx, stream);
 }
 
 h3q_status h3q_prepare_weight(const float* w, int64_t N, int64_t K, int8_t* wq, float* sw, cudaStream_t stream) {
@@ -257,8 +288,7 @@ h3q_status h3q_prepare_weight(const float* w, int64_t N, int64_t K, int8_t* wq, 
   if (N == 0) return H3Q_OK;
   if (!w || !wq || !sw || !aligned16(w) || !aligned16(wq) || !aligned16(sw)) return H3Q_ERR_INVALID_ARG;
   if (K > H3Q_MAX_K || N > INT32_MAX) return H3Q_ERR_UNSUPPORTED;
-  const cudaError_t e = h3q::launch_rotquant(w, N, K, wq, sw, g_wait_limit_ns.load(), stream);
-  return e == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+  return run_rotquant(w, N, K, wq, sw, stream);
 }
 
 h3q_status h3q_linear_w8a8(const int8_t* xq, const float* sx, int64_t M, int64_t K, const int8_t* wq,

@@ -3,40 +3,47 @@
 // (per-token) absmax int8 quantization.
 //
 // Data movement: a persistent grid; in each block one producer thread streams
-// work items (R whole rows, contiguous in memory) into a ring of shared-memory
-// stages with 1D bulk copies (cp.async.bulk, completion on an mbarrier), so
-// several items are in flight per block while the consumer warps work. Each row
-// is read from HBM once and its codes are written once.
+// work items (R whole rows) into a ring of shared-memory stages with TMA tensor
+// copies (a 3D view of the rows as 128-byte units, 128-byte swizzle, completion
+// on an mbarrier), so several items are in flight per block while the consumer
+// warps work. Each row is read from HBM once and its codes are written once.
 //
-// Rotation of one 256-group by a half-warp (16 lanes), seen as a 16 x 16 matrix
-// X[a][b] = x[16a + b]:
-//   phase A  lane a holds row a (16 contiguous elements) and applies the
-//            butterflies of index bits 0-3 in registers;
-//   transpose through a per-half-warp shared-memory scratch (fp32, chunks
-//            swizzled so both the row writes and the column reads are free of
-//            bank conflicts);
-//   phase B  lane b holds column b and applies the butterflies of bits 4-7.
-// Each phase keeps its 16 values as packed pairs (v[r], v[r+8]) and runs three
-// stages on the sm_100 two-wide fp32 add and the fourth inside each pair. The
-// bits are processed in ascending order and every butterfly is one correctly
-// rounded fp32 add or subtract, so each rotated value has the same bits as the
-// pairwise-tree sum of the explicit H/16 product. No shuffle is needed. The
-// 1/16 moves to the scale: y16 = 16 y and s16 = max|y16| / 127 = 16 s exactly,
-// and y16 / s16 = y / s, so the codes are unchanged.
+// Rotation of one 256-group by a quarter-warp (8 lanes), seen as an 8 x 32
+// matrix X[j][m] = x[32 j + m]:
+//   phase A  lane j holds row j (32 contiguous elements) and applies the
+//            butterflies of index bits 0-4 in registers. Its 16-byte chunks are
+//            read from the swizzled stage, so the 8 lanes of a quarter hit 8
+//            different bank quads;
+//   transpose through a per-quarter fp32 scratch of 8 rows with a 144-byte pitch
+//            (each row shifted by one bank quad), written and read in 16-byte
+//            pieces without bank conflicts;
+//   phase B  lane l holds elements 32 j + 4 l + i (j = 0..7, i = 0..3) and
+//            applies the butterflies of bits 5-7.
+// Values are kept as pairs (v[2i], v[2i+1]): bit 0 is one scalar add and one
+// scalar subtract per pair (fused with the bf16 unpacking), every other bit runs
+// on the sm_100 two-wide fp32 add and FMA. The bits are processed in ascending
+// order and every butterfly is one correctly rounded fp32 add or subtract, so
+// each rotated value has the same bits as the pairwise-tree sum of the explicit
+// H/16 product. The 1/16 moves to the scale: y16 = 16 y and s16 = max|y16| / 127
+// = 16 s exactly, and y16 / s16 = y / s, so the codes are unchanged.
 //
 // Quantization needs rne(RN(y / s)) per element. Each row gets rs = RN(1/s)
-// once; each quotient is q0 = RN(y rs) refined twice with exact FMA residuals,
-// e = y - q s, q <- RN(q + e rs) (Markstein, "Computation of elementary
-// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
-// 1990): after the first step q is within one ulp of y/s, and the second step
-// returns the correctly rounded quotient. Rows whose scale is below 2^-100 are
-// first rescaled by 2^64 (exact). The integer is read from the bits
-// of q + 1.5*2^23, whose add rounds half to even; its low byte is the int8 code.
-// |y| <= max|y| bounds y/s by 127 (1 + 2^-23), so no clamp is needed. The codes
-// of a column are scattered bytes of the group; they pass through the slot's
-// shared buffer and leave as one 16-byte store per lane.
+// once. A candidate integer n = rne(y rs) and its exact-sign residual y - n s
+// decide the code for all values but those within about 2^-16 of a half-integer
+// quotient; for those the quotient is q0 = RN(y rs) refined twice with exact FMA
+// residuals, e = y - q s, q <- RN(q + e rs) (Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev.
+// 34(1), 1990): after the first step q is within one ulp of y/s, and the second
+// step returns the correctly rounded quotient, then rounded half to even. Rows
+// whose scale is below 2^-100 are first rescaled by 2^64 (exact). Integers are
+// read from the bits of a value plus 1.5*2^23, whose low byte is the int8 code.
+// |y| <= max|y| bounds y/s by 127 (1 + 2^-23), so no clamp is needed. In phase B
+// a lane's codes for j come from four consecutive elements: three byte permutes
+// make one 32-bit word, stored straight to the row (a quarter writes 32
+// contiguous bytes per j).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -45,96 +52,130 @@
 namespace h3q {
 
 constexpr int kRqMaxRows = 16;
-constexpr int kRqSlotBytes = 1024 + 64;  // per half-warp: 16 x 16 fp32 scratch + 64 B so slots shift banks by 16
+constexpr int kRqRowPitch = 144;                  // scratch row: 32 fp32 + 16 bytes
+constexpr int kRqScratchBytes = 8 * kRqRowPitch;  // per quarter-warp
+constexpr int kRqMaxWarps = 31;                   // consumer warps per block
 
+// 16-byte shared-memory load at a shared-window address (ordered after the
+// stage's mbarrier wait, which is also a volatile asm statement).
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// 3D tiled load of one box, completion counted on `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap* map, uint64_t* bar, int32_t x,
+                                            int32_t y, int32_t z, uint64_t cache_policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(cache_policy)
+      : "memory");
+}
+
+// Phase A input: lane's 32 elements (32 j .. 32 j + 31 of its group) from the
+// swizzled stage, chunk k at address a ^ (16 k), with the bit-0 butterfly:
+// on return p[i] = (v[2i] + v[2i+1], v[2i] - v[2i+1]).
 template <typename T>
-struct Row16;  // lane a's 16 contiguous elements 16a .. 16a+15 of a group, as pairs (v[r], v[r+8])
+struct LaneLoad;
 
 template <>
-struct Row16<__nv_bfloat16> {
-  static __device__ __forceinline__ void load(const __nv_bfloat16* grp, int a, float2 (&p)[8]) {
-    const uint4* row = reinterpret_cast<const uint4*>(grp + 16 * a);
-    const uint4 lo = row[0], hi = row[1];  // elements 0-7 and 8-15
-    const uint32_t ul[4] = {lo.x, lo.y, lo.z, lo.w}, uh[4] = {hi.x, hi.y, hi.z, hi.w};
+struct LaneLoad<__nv_bfloat16> {
+  static constexpr int kChunks = 4;  // 8 elements per 16-byte chunk
+  static __device__ __forceinline__ void load(uint32_t a, float2 (&p)[16]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {  // element 2i of a word is its low half
-      p[2 * i] = make_float2(__uint_as_float(ul[i] << 16), __uint_as_float(uh[i] << 16));
-      p[2 * i + 1] = make_float2(__uint_as_float(ul[i] & 0xFFFF0000u), __uint_as_float(uh[i] & 0xFFFF0000u));
-    }
-  }
-};
-
-template <>
-struct Row16<float> {
-  static __device__ __forceinline__ void load(const float* grp, int a, float2 (&p)[8]) {
-    const float4* row = reinterpret_cast<const float4*>(grp + 16 * a);
-    const float4 c0 = row[0], c1 = row[1], c2 = row[2], c3 = row[3];
-    p[0] = make_float2(c0.x, c2.x); p[1] = make_float2(c0.y, c2.y);
-    p[2] = make_float2(c0.z, c2.z); p[3] = make_float2(c0.w, c2.w);
-    p[4] = make_float2(c1.x, c3.x); p[5] = make_float2(c1.y, c3.y);
-    p[6] = make_float2(c1.z, c3.z); p[7] = make_float2(c1.w, c3.w);
-  }
-};
-
-// Unnormalized 16-point Walsh-Hadamard transform of v[0..15] held as
-// p[r] = (v[r], v[r+8]): bits 0-2 on packed pairs, then bit 3 inside each pair.
-__device__ __forceinline__ void fwht16(float2 (&p)[8]) {
-  const float2 minus1 = make_float2(-1.0f, -1.0f);
+    for (int k = 0; k < 4; ++k) {
+      const uint4 w = lds128(a ^ (16u * k));
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int b = 0; b < 3; ++b) {
-    const int s = 1 << b;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      if ((r & s) == 0) {
-        const float2 lo = p[r], hi = p[r + s];
-        p[r] = __fadd2_rn(lo, hi);
-        p[r + s] = __ffma2_rn(hi, minus1, lo);  // lo - hi, one rounding
+      for (int i = 0; i < 4; ++i) {  // element 2i of a word is its low half
+        const float lo = __uint_as_float(__byte_perm(u[i], 0u, 0x1044)), hi = __uint_as_float(u[i] & 0xFFFF0000u);
+        p[4 * k + i] = make_float2(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
       }
     }
   }
+};
+
+template <>
+struct LaneLoad<float> {
+  static constexpr int kChunks = 8;  // 4 elements per 16-byte chunk
+  static __device__ __forceinline__ void load(uint32_t a, float2 (&p)[16]) {
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const float lo = p[r].x, hi = p[r].y;
-    p[r] = make_float2(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
+    for (int k = 0; k < 8; ++k) {
+      const uint4 w = lds128(a ^ (16u * k));
+      const float v0 = __uint_as_float(w.x), v1 = __uint_as_float(w.y), v2 = __uint_as_float(w.z),
+                  v3 = __uint_as_float(w.w);
+      p[2 * k] = make_float2(__fadd_rn(v0, v1), __fsub_rn(v0, v1));
+      p[2 * k + 1] = make_float2(__fadd_rn(v2, v3), __fsub_rn(v2, v3));
+    }
+  }
+};
+
+// Butterflies over pair indices: for every i with bit b clear,
+// (p[i], p[i + 2^b]) <- (p[i] + p[i + 2^b], p[i] - p[i + 2^b]), bits B0..B1-1 in
+// ascending order, each a two-wide correctly rounded add or subtract. `stride`
+// maps a butterfly index to the pair index (phase B interleaves two pairs per j).
+template <int N, int B0, int B1, int STRIDE>
+__device__ __forceinline__ void butterflies(float2 (&p)[N]) {
+  const float2 minus1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+  for (int b = B0; b < B1; ++b) {
+    const int s = 1 << b;
+#pragma unroll
+    for (int i = 0; i < N / STRIDE; ++i) {
+      if ((i & s) == 0) {
+#pragma unroll
+        for (int h = 0; h < STRIDE; ++h) {
+          const float2 lo = p[STRIDE * i + h], hi = p[STRIDE * (i + s) + h];
+          p[STRIDE * i + h] = __fadd2_rn(lo, hi);
+          p[STRIDE * (i + s) + h] = __ffma2_rn(hi, minus1, lo);  // lo - hi, one rounding
+        }
+      }
+    }
   }
 }
 
-// Scratch layout: row a holds 16 fp32 values; its 16-byte chunk k sits at chunk
-// position k ^ ((a >> 1) & 3) of the row.
-// Rotates one group: on return, p[r] = (y16[16 r + b], y16[16 (r + 8) + b]) for
-// this lane's column b = hl. `scratch` is the half-warp's private fp32 area.
-template <typename T>
-__device__ __forceinline__ void rotate_group(const T* grp, int hl, float* scratch, float2 (&p)[8]) {
-  Row16<T>::load(grp, hl, p);
-  fwht16(p);  // index bits 0-3
-  const int sw = (hl >> 1) & 3;
+// Rotates one group whose lane values (after the bit-0 butterfly, as loaded by
+// LaneLoad) are in p; `scr` is the quarter's scratch and `l` the lane within the
+// quarter. On return p[2j + h] = (y16[32 j + 4 l + 2h], y16[32 j + 4 l + 2h + 1]).
+__device__ __forceinline__ void rotate_group(float* scr, int l, float2 (&p)[16]) {
+  butterflies<16, 0, 4, 1>(p);  // index bits 1-4
+  float* row = scr + (kRqRowPitch / 4) * l;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {  // row hl, chunk k = elements 4k .. 4k+3
-    const float4 c = k < 2 ? make_float4(p[4 * k].x, p[4 * k + 1].x, p[4 * k + 2].x, p[4 * k + 3].x)
-                           : make_float4(p[4 * k - 8].y, p[4 * k - 7].y, p[4 * k - 6].y, p[4 * k - 5].y);
-    *reinterpret_cast<float4*>(scratch + 16 * hl + 4 * (k ^ sw)) = c;
-  }
+  for (int k = 0; k < 8; ++k)  // elements 4k .. 4k+3 of row l
+    *reinterpret_cast<float4*>(row + 4 * k) = make_float4(p[2 * k].x, p[2 * k].y, p[2 * k + 1].x, p[2 * k + 1].y);
   __syncwarp();
-  // column hl: row r's element sits at 16 r + 4 ((hl >> 2) ^ (r >> 1) & 3) + (hl & 3);
-  // four base pointers (one per value of r >> 1 & 3) leave an immediate offset per row
-  const float* col = scratch + (hl & 3);
-  const int x = hl >> 2;
-  const float* b0 = col + 4 * (x & 3);
-  const float* b1 = col + 4 * ((x ^ 1) & 3);
-  const float* b2 = col + 4 * ((x ^ 2) & 3);
-  const float* b3 = col + 4 * ((x ^ 3) & 3);
-  const float* base[4] = {b0, b1, b2, b3};
 #pragma unroll
-  for (int r = 0; r < 8; ++r) p[r] = make_float2(base[(r >> 1) & 3][16 * r], base[((r + 8) >> 1) & 3][16 * (r + 8)]);
-  __syncwarp();  // the scratch is rewritten next (codes or the next group)
-  fwht16(p);     // index bits 4-7
+  for (int j = 0; j < 8; ++j) {  // elements 4l .. 4l+3 of row j
+    const float4 c = *reinterpret_cast<const float4*>(scr + (kRqRowPitch / 4) * j + 4 * l);
+    p[2 * j] = make_float2(c.x, c.y);
+    p[2 * j + 1] = make_float2(c.z, c.w);
+  }
+  __syncwarp();                 // the scratch is rewritten by the next group
+  butterflies<16, 0, 3, 2>(p);  // index bits 5-7
 }
 
-// max of three fp32 values (sm_100 three-input max).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
+// max(m, |a|, |b|) (sm_100 three-input max; the absolute values are taken in
+// the same asm block so they fold into the max's operands).
+__device__ __forceinline__ float fmax_abs2(float m, float a, float b) {
   float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  asm("{\n\t.reg .f32 aa, ab;\n\tabs.f32 aa, %2;\n\tabs.f32 ab, %3;\n\tmax.f32 %0, %1, aa, ab;\n\t}"
+      : "=f"(r)
+      : "f"(m), "f"(a), "f"(b));
   return r;
+}
+
+__device__ __forceinline__ float group_lane_absmax(const float2 (&p)[16]) {
+  float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    m0 = fmax_abs2(m0, p[i].x, p[i].y);
+    m1 = fmax_abs2(m1, p[i + 1].x, p[i + 1].y);
+  }
+  return fmaxf(m0, m1);
 }
 
 // Per-row quotient constants: y / s is formed as (y f) / (s f) with f = 2^64 for
@@ -162,63 +203,111 @@ __device__ __forceinline__ RowQuot row_quotient(float s16) {
   return r;
 }
 
-// int8 codes rne(y16 / s16) of this lane's column hl, written as bytes into the
-// group's 256-byte code buffer at element positions 16 r + hl and 16 (r + 8) + hl.
-// kRescaled: the row's f is 2^64 (scale below 2^-100); otherwise f = 1 and the exact
-// rescaling is skipped.
+// int8 codes rne(RN(y16 / s16)) of this lane's 32 values, stored as one 32-bit
+// word per j at out + 32 j (out = the row's codes + 256 g + 4 l).
+//
+// Fast path, three fp32 operations per value: the candidate n = rne(y rs) comes
+// from one FMA onto 1.5*2^23 (whose bits then hold n in the low byte), and the
+// residual r = RN(y - n s) from another. With t = RN(s (1/2 - 2^-16)), |r| <= t
+// bounds |y/s - n| below 1/2 - 2^-16 + 2^-24; RN(y/s) moves y/s by at most 2^-18
+// (|y/s| < 128), so n is the integer nearest RN(y/s) and the code is exact. A lane
+// whose largest |r| exceeds t (y/s within about 2^-16 of a half-integer, some
+// 3e-5 of the values) recomputes its 32 quotients as correctly rounded IEEE
+// quotients (two Markstein steps) and rounds those. kRescaled: the row's f is
+// 2^64 (scale below 2^-100); otherwise f = 1 and the exact rescaling is skipped.
+// An all-zero row has s = 0, rs = 0, t = 0 and residuals 0: codes 0.
 template <bool kRescaled>
-__device__ __forceinline__ void quantize_column(const float2 (&p)[8], const RowQuot& rq, int hl,
-                                                uint8_t* codes) {
-  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+__device__ __forceinline__ void quantize_store(const float2 (&p)[16], const RowQuot& rq, int8_t* out) {
+  const float2 magic = make_float2(12582912.0f, 12582912.0f), nmagic = make_float2(-12582912.0f, -12582912.0f);
   const float2 f2 = make_float2(rq.f, rq.f), r2 = make_float2(rq.rs, rq.rs), ns2 = make_float2(-rq.sf, -rq.sf);
+  const float t = __fmul_rn(rq.sf, 0.4999847412109375f);  // 1/2 - 2^-16
+  float2 u[16];
+  float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const float2 y = kRescaled ? __fmul2_rn(p[r], f2) : p[r];  // exact
-    float2 q = __fmul2_rn(y, r2);
-    float2 e = __ffma2_rn(q, ns2, y);
-    q = __ffma2_rn(e, r2, q);
-    e = __ffma2_rn(q, ns2, y);
-    q = __ffma2_rn(e, r2, q);
-    const float2 u = __fadd2_rn(q, magic);
-    codes[16 * r + hl] = static_cast<uint8_t>(__float_as_uint(u.x));
-    codes[16 * (r + 8) + hl] = static_cast<uint8_t>(__float_as_uint(u.y));
+  for (int i = 0; i < 16; ++i) {
+    const float2 y = kRescaled ? __fmul2_rn(p[i], f2) : p[i];  // exact
+    u[i] = __ffma2_rn(y, r2, magic);
+    const float2 r = __ffma2_rn(__fadd2_rn(u[i], nmagic), ns2, y);
+    if (i & 1)
+      m1 = fmax_abs2(m1, r.x, r.y);
+    else
+      m0 = fmax_abs2(m0, r.x, r.y);
+  }
+  if (fmaxf(m0, m1) > t) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 y = kRescaled ? __fmul2_rn(p[i], f2) : p[i];
+      float2 q = __fmul2_rn(y, r2);
+      float2 e = __ffma2_rn(q, ns2, y);
+      q = __ffma2_rn(e, r2, q);
+      e = __ffma2_rn(q, ns2, y);
+      q = __ffma2_rn(e, r2, q);
+      u[i] = __fadd2_rn(q, magic);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t lo = __byte_perm(__float_as_uint(u[2 * j].x), __float_as_uint(u[2 * j].y), 0x0040);
+    const uint32_t hi = __byte_perm(__float_as_uint(u[2 * j + 1].x), __float_as_uint(u[2 * j + 1].y), 0x0040);
+    *reinterpret_cast<uint32_t*>(out + 32 * j) = __byte_perm(lo, hi, 0x5410);
   }
 }
 
 struct RqArgs {
-  int64_t M;          // rows
-  int K;              // row length (multiple of 256)
-  int R;              // rows per work item
-  int64_t items;      // ceil(M / R)
-  int stages;         // shared-memory ring depth
-  uint32_t stage_bytes;
+  int64_t M;             // rows
+  int K;                 // row length (multiple of 256)
+  int R;                 // rows per work item
+  int64_t items;         // ceil(M / R)
+  int stages;            // shared-memory ring depth
+  uint32_t stage_bytes;  // copies * copy_bytes
+  uint32_t copy_bytes;   // shared-memory room of one TMA box, its bytes rounded up to 1024
+  uint32_t tx_bytes;     // bytes the item's boxes deliver: copies x R x units_per_copy x 128
+  int copies;            // TMA boxes per item (the row split along K)
+  int units_per_copy;    // 128-byte units of a row in one box
   int8_t* q;
   float* s_out;
   uint64_t wait_limit_ns;
 };
 
 struct RqShape {
-  int gps, warps, rows, stages;  // groups per half-warp slot, consumer warps, rows per item, ring depth
-  bool small;                    // built for three blocks per SM
+  int gps, warps, rows, stages;  // groups per quarter-warp, consumer warps, rows per item, ring depth
 };
 
 inline size_t rotquant_smem_bytes(int stages, uint32_t stage_bytes, int warps) {
-  return size_t(stages) * stage_bytes + size_t(2 * warps) * kRqSlotBytes + 2 * sizeof(uint64_t) * stages +
+  return 1024 + size_t(stages) * stage_bytes + size_t(4 * warps) * kRqScratchBytes + 2 * sizeof(uint64_t) * stages +
          3 * kRqMaxRows * 4 + 16;
 }
 
-// Warp 0 is the producer; warps 1..W are consumers with 2W half-warp slots, each
-// taking GPS groups per item: 2 * W * GPS >= R * (K / 256). SMALL builds for
-// blocks of at most 16 warps, three per SM (40 registers); otherwise up to 32
-// warps, one per SM.
-template <typename T, int GPS, bool SMALL>
-__global__ void __launch_bounds__(SMALL ? 512 : (GPS == 1 ? 1024 : 544), SMALL ? 3 : 1)
-    rotquant_kernel(const T* __restrict__ x, const RqArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
+// Byte offset, inside a stage, of the first 16-byte chunk of the 32 elements
+// 32 l .. 32 l + 31 of group g in row r of the item: the stage holds `copies`
+// boxes of copy_bytes; box c covers the units [c U, (c + 1) U) of every row as
+// [rows][U][128 bytes], chunk x of unit n stored at chunk x ^ (n & 7).
+template <typename T>
+__device__ __forceinline__ uint32_t lane_tile_offset(const RqArgs& a, int r, int g, int l) {
+  constexpr int kPerUnit = 128 / int(sizeof(T));
+  const int e0 = 256 * g + 32 * l;
+  const int unit = e0 / kPerUnit;
+  const int chunk = (e0 % kPerUnit) * int(sizeof(T)) / 16;
+  const int c = unit / a.units_per_copy, un = unit - c * a.units_per_copy;
+  const int n = r * a.units_per_copy + un;
+  return uint32_t(c) * a.copy_bytes + 128u * uint32_t(n) + 16u * uint32_t(chunk ^ (n & 7));
+}
+
+// Warp 0 is the producer; warps 1..W are consumers with 4W quarter-warps, each
+// taking GPS groups per item: 4 W GPS >= R (K / 256).
+template <typename T, int GPS>
+__global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
+    rotquant_kernel(const __grid_constant__ CUtensorMap tmap, const RqArgs a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+  uint8_t* smem = smem_raw + pad;  // 1024-byte aligned: stages, then scratch
+  const uint32_t stage0 = raw + pad;
   const int n_cons = blockDim.x - 32;
-  const int HW = n_cons >> 4;
-  uint8_t* scratch_base = smem + size_t(a.stages) * a.stage_bytes;  // HW slots of kRqSlotBytes
-  uint64_t* full = reinterpret_cast<uint64_t*>(scratch_base + size_t(HW) * kRqSlotBytes);
+  const int NQ = n_cons >> 3;
+  float* scratch_base = reinterpret_cast<float*>(smem + size_t(a.stages) * a.stage_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scratch_base) +
+                                               size_t(NQ) * kRqScratchBytes);
   uint64_t* empty = full + a.stages;
   uint32_t* row_amax = reinterpret_cast<uint32_t*>(empty + a.stages);  // [3][kRqMaxRows]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(row_amax + 3 * kRqMaxRows);
@@ -240,6 +329,7 @@ __global__ void __launch_bounds__(SMALL ? 512 : (GPS == 1 ? 1024 : 544), SMALL ?
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
+      tma_prefetch_desc(&tmap);
       const uint64_t pol = policy_evict_first();
       int stage = 0;
       uint32_t phase = 0;
@@ -250,11 +340,11 @@ __global__ void __launch_bounds__(SMALL ? 512 : (GPS == 1 ? 1024 : 544), SMALL ?
           ok = false;
           break;
         }
-        const int64_t row0 = item * a.R;
-        const int64_t nrows = (a.M - row0) < a.R ? (a.M - row0) : a.R;
-        const uint32_t bytes = static_cast<uint32_t>(nrows * a.K * int64_t(sizeof(T)));
-        mbar_arrive_expect_tx(&full[stage], bytes);
-        bulk_load(smem + size_t(stage) * a.stage_bytes, x + row0 * a.K, bytes, &full[stage], pol);
+        mbar_arrive_expect_tx(&full[stage], a.tx_bytes);
+        const uint32_t dst = stage0 + uint32_t(stage) * a.stage_bytes;
+        for (int c = 0; c < a.copies; ++c)
+          tma_load_3d(dst + uint32_t(c) * a.copy_bytes, &tmap, &full[stage], 0, c * a.units_per_copy,
+                      static_cast<int32_t>(item * a.R), pol);
         ++issued;
         if (++stage == a.stages) {
           stage = 0;
@@ -274,18 +364,19 @@ __global__ void __launch_bounds__(SMALL ? 512 : (GPS == 1 ? 1024 : 544), SMALL ?
 
   // ------------------------------------------------------------------ consumers
   const int c = threadIdx.x - 32;
-  const int hl = c & 15;
-  const int slot = c >> 4;
-  float* scratch = reinterpret_cast<float*>(scratch_base + size_t(slot) * kRqSlotBytes);
-  uint8_t* codes_buf = reinterpret_cast<uint8_t*>(scratch);  // reused once the group is rotated
+  const int l = c & 7;
+  const int qd = c >> 3;
+  float* scr = scratch_base + size_t(qd) * (kRqScratchBytes / 4);
   int rr[GPS], gg[GPS];
   bool act[GPS];
+  uint32_t toff[GPS];
 #pragma unroll
   for (int t = 0; t < GPS; ++t) {
-    const int i = t * HW + slot;
+    const int i = t * NQ + qd;
     act[t] = i < a.R * G;
     rr[t] = act[t] ? i / G : 0;
     gg[t] = act[t] ? i - rr[t] * G : 0;
+    toff[t] = lane_tile_offset<T>(a, rr[t], gg[t], l);
   }
 
   // Row slot buffers of the absmax: item k uses buffer k % 3; buffer (k + 1) % 3,
@@ -293,86 +384,108 @@ __global__ void __launch_bounds__(SMALL ? 512 : (GPS == 1 ? 1024 : 544), SMALL ?
   // k + 1's atomics.
   int stage = 0;
   uint32_t phase = 0;
-  for (int64_t item = blockIdx.x, it = 0; item < a.items; item += gridDim.x, ++it) {
+  int buf = 0, next = kRqMaxRows;  // offsets of buffers it % 3 and (it + 1) % 3
+  for (int64_t item = blockIdx.x; item < a.items; item += gridDim.x) {
     mbar_wait_bounded(&full[stage], phase, a.wait_limit_ns, abort_flag);  // on expiry: garbage, no hang
-    const T* tile = reinterpret_cast<const T*>(smem + size_t(stage) * a.stage_bytes);
-    const int buf = static_cast<int>(it % 3);
-    if (c < kRqMaxRows) row_amax[((it + 1) % 3) * kRqMaxRows + c] = 0u;
+    const uint32_t tile = stage0 + uint32_t(stage) * a.stage_bytes;
+    if (c < kRqMaxRows) row_amax[next + c] = 0u;
     const int64_t row0 = item * a.R;
 
-    float2 p[GPS][8];
+    float2 p[GPS][16];
 #pragma unroll
-    for (int t = 0; t < GPS; ++t) {
-      rotate_group(tile + rr[t] * a.K + gg[t] * 256, hl, scratch, p[t]);
-      float m = 0.0f;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) m = fmax3(m, fabsf(p[t][r].x), fabsf(p[t][r].y));
-#pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-      if (hl == 0 && act[t] && row0 + rr[t] < a.M)
-        atomicMax(&row_amax[buf * kRqMaxRows + rr[t]], __float_as_uint(m));
-    }
-    mbar_arrive(&empty[stage]);  // this thread's reads of the stage are done
+    for (int t = 0; t < GPS; ++t) LaneLoad<T>::load(tile + toff[t], p[t]);
+    mbar_arrive(&empty[stage]);  // this thread's reads of the stage are done: the producer may refill it
     if (++stage == a.stages) {
       stage = 0;
       phase ^= 1u;
+    }
+#pragma unroll
+    for (int t = 0; t < GPS; ++t) {
+      rotate_group(scr, l, p[t]);
+      float m = group_lane_absmax(p[t]);
+#pragma unroll
+      for (int o = 1; o <= 4; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if (l == 0 && act[t] && row0 + rr[t] < a.M) atomicMax(&row_amax[buf + rr[t]], __float_as_uint(m));
     }
     named_barrier(1, n_cons);
 #pragma unroll
     for (int t = 0; t < GPS; ++t) {
       const int64_t row = row0 + rr[t];
-      const float am = __uint_as_float(row_amax[buf * kRqMaxRows + rr[t]]);
+      const float am = __uint_as_float(row_amax[buf + rr[t]]);
       const float s16 = div127(am);
-      if (hl == 0 && gg[t] == 0 && act[t] && row < a.M) a.s_out[row] = __fmul_rn(s16, 0.0625f);
-      const RowQuot rq = row_quotient(s16);
-      if (rq.f == 1.0f)
-        quantize_column<false>(p[t], rq, hl, codes_buf);
-      else
-        quantize_column<true>(p[t], rq, hl, codes_buf);
-      __syncwarp();
-      const uint4 out = *reinterpret_cast<const uint4*>(codes_buf + 16 * hl);  // elements 16 hl .. 16 hl + 15
-      __syncwarp();  // before the buffer is reused
-      if (act[t] && row < a.M) *reinterpret_cast<uint4*>(a.q + row * a.K + gg[t] * 256 + 16 * hl) = out;
+      if (l == 0 && gg[t] == 0 && act[t] && row < a.M) a.s_out[row] = __fmul_rn(s16, 0.0625f);
+      if (act[t] && row < a.M) {
+        const RowQuot rq = row_quotient(s16);
+        int8_t* out = a.q + row * a.K + 256 * gg[t] + 4 * l;
+        if (rq.f == 1.0f)
+          quantize_store<false>(p[t], rq, out);
+        else
+          quantize_store<true>(p[t], rq, out);
+      }
     }
+    buf = next;
+    next = next == 2 * kRqMaxRows ? 0 : next + kRqMaxRows;
   }
 }
 
 // ----------------------------------------------------------------------------
 // Host side: shape choice and launch.
 
-template <typename T, int GPS, bool SMALL>
+template <typename T, int GPS>
 cudaError_t rotquant_prepare_attr(int dev) {
   static bool done[16] = {};
   if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
   if (done[dev]) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(rotquant_kernel<T, GPS, SMALL>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  const cudaError_t e =
+      cudaFuncSetAttribute(rotquant_kernel<T, GPS>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   if (e == cudaSuccess) done[dev] = true;
   return e;
 }
 
-template <typename T, int GPS, bool SMALL>
-int rotquant_occupancy_t(int threads, size_t smem, int dev) {
-  if (rotquant_prepare_attr<T, GPS, SMALL>(dev) != cudaSuccess) return 0;
+template <typename T>
+int rotquant_occupancy(int gps, int threads, size_t smem, int dev) {
   int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotquant_kernel<T, GPS, SMALL>, threads, smem) !=
-      cudaSuccess)
-    return 0;
+  if (gps == 1) {
+    if (rotquant_prepare_attr<T, 1>(dev) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotquant_kernel<T, 1>, threads, smem) != cudaSuccess)
+      return 0;
+  } else {
+    if (rotquant_prepare_attr<T, 2>(dev) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotquant_kernel<T, 2>, threads, smem) != cudaSuccess)
+      return 0;
+  }
   return occ;
 }
 
+// TMA boxes per item and 128-byte units per box for rows of K elements of T: a
+// box dimension holds at most 256 units.
 template <typename T>
-int rotquant_occupancy(int gps, bool small, int threads, size_t smem, int dev) {
-  if (gps == 1) return small ? rotquant_occupancy_t<T, 1, true>(threads, smem, dev)
-                             : rotquant_occupancy_t<T, 1, false>(threads, smem, dev);
-  return small ? rotquant_occupancy_t<T, 2, true>(threads, smem, dev)
-               : rotquant_occupancy_t<T, 2, false>(threads, smem, dev);
+inline void rotquant_copies(int K, int* copies, int* units_per_copy) {
+  const int units = K * int(sizeof(T)) / 128;
+  int n = (units + 255) / 256;
+  while (units % n != 0) ++n;
+  *copies = n;
+  *units_per_copy = units / n;
 }
 
-// For a row of G groups: among shapes with 1 or 2 groups per slot, up to 8 rows
-// per item and 2 to 6 stages, keep the one with the most consumer warps doing
-// useful work per SM (occupancy times the share of busy slots), then the most
-// loads in flight per SM (up to 128 KB).
+inline uint32_t align1024(uint64_t x) { return static_cast<uint32_t>((x + 1023u) & ~uint64_t(1023u)); }
+
+template <typename T>
+inline uint32_t rotquant_copy_bytes(int K, int R) {
+  int n = 0, u = 0;
+  rotquant_copies<T>(K, &n, &u);
+  return align1024(uint64_t(R) * u * 128u);
+}
+
+// For a row of G groups: among shapes with 1 or 2 groups per quarter-warp, up to
+// 8 rows per item and 2 to 6 stages, keep the one with the most consumer warps
+// doing useful work per SM (occupancy times the share of busy quarters), then the
+// most loads in flight per SM (up to 128 KB). bf16 rows of the model's widths use
+// the shapes measured fastest on B200 at 16384 rows (two blocks per SM, two
+// stages each): K = 5376: one group per quarter, 11 consumer warps, 2 rows per
+// item (3.28 TB/s); K = 10752: one group per quarter, 11 warps, one row per item
+// (3.5 TB/s); K = 14336: two groups per quarter, 7 warps, one row per item
+// (3.7 TB/s).
 template <typename T>
 RqShape rotquant_plan(int K, int dev, int* blocks_per_sm) {
   static RqShape cache[16][65] = {};
@@ -382,18 +495,15 @@ RqShape rotquant_plan(int K, int dev, int* blocks_per_sm) {
     *blocks_per_sm = cache_occ[dev][G];
     return cache[dev][G];
   }
-  RqShape best{0, 0, 0, 0, false};
+  RqShape best{0, 0, 0, 0};
   int best_occ = 0;
   double best_score = -1.0;
-  // Shapes measured fastest on B200 (bf16 rows, M = 16384): K = 5376: 2 groups per
-  // slot, 3 rows per item, 16 consumer warps, 4 stages (2.92 TB/s, against 2.57 for
-  // the best one-group shape); rows of 32 to 62 groups: one group per slot, one row
-  // per item, ceil(G / 2) consumer warps, 4 stages (K = 14336: 28 warps, 2.95 TB/s;
-  // K = 10752: 21 warps, 2.56 TB/s against 2.05 for the planner's choice).
-  if (sizeof(T) == 2 && (K == 5376 || (G >= 32 && G <= 62))) {
-    const RqShape pick = K == 5376 ? RqShape{2, 16, 3, 4, false} : RqShape{1, (G + 1) / 2, 1, 4, false};
-    const uint32_t stage_bytes = static_cast<uint32_t>(int64_t(pick.rows) * K * int64_t(sizeof(T)));
-    const int occ = rotquant_occupancy<T>(pick.gps, pick.small, 32 * (pick.warps + 1),
+  if (sizeof(T) == 2 && (G == 21 || G == 42 || G == 56)) {
+    const RqShape pick = G == 21 ? RqShape{1, 11, 2, 2} : G == 42 ? RqShape{1, 11, 1, 2} : RqShape{2, 7, 1, 2};
+    int n = 0, u = 0;
+    rotquant_copies<T>(K, &n, &u);
+    const uint32_t stage_bytes = uint32_t(n) * rotquant_copy_bytes<T>(K, pick.rows);
+    const int occ = rotquant_occupancy<T>(pick.gps, 32 * (pick.warps + 1),
                                           rotquant_smem_bytes(pick.stages, stage_bytes, pick.warps), dev);
     if (occ >= 1) {
       best = pick;
@@ -402,30 +512,30 @@ RqShape rotquant_plan(int K, int dev, int* blocks_per_sm) {
     }
   }
   for (int gps = 1; gps <= 2 && best_score < 1e29; ++gps)
-    for (int R = 1; R <= 8 && R <= kRqMaxRows; ++R)
-      for (int small = 1; small >= 0; --small) {
-        const int slots = R * G;
-        const int W = (slots + 2 * gps - 1) / (2 * gps);
-        const int threads = 32 * (W + 1);
-        if (threads > (small ? 512 : (gps == 1 ? 1024 : 544))) continue;
-        const uint32_t stage_bytes = static_cast<uint32_t>(int64_t(R) * K * int64_t(sizeof(T)));
-        for (int stages = 2; stages <= 6; ++stages) {
-          const size_t smem = rotquant_smem_bytes(stages, stage_bytes, W);
-          if (smem > 227 * 1024) break;
-          const int occ = rotquant_occupancy<T>(gps, small != 0, threads, smem, dev);
-          if (occ < 1) break;
-          // useful consumer warps per SM, then loads in flight per SM (capped)
-          const double busy = double(slots) / double(2 * W * gps);
-          const double inflight = double(occ) * stages * stage_bytes;
-          const double score = occ * W * busy + 4.0 * (inflight < 131072.0 ? inflight : 131072.0) / 131072.0 -
-                               0.01 * gps - 0.001 * R;
-          if (score > best_score) {
-            best_score = score;
-            best = {gps, W, R, stages, small != 0};
-            best_occ = occ;
-          }
+    for (int R = 1; R <= 8 && R <= kRqMaxRows; ++R) {
+      const int slots = R * G;
+      const int W = (slots + 4 * gps - 1) / (4 * gps);
+      const int threads = 32 * (W + 1);
+      if (W > kRqMaxWarps || threads > (gps == 1 ? 768 : 512)) continue;
+      int n = 0, u = 0;
+      rotquant_copies<T>(K, &n, &u);
+      const uint32_t stage_bytes = uint32_t(n) * rotquant_copy_bytes<T>(K, R);
+      for (int stages = 2; stages <= 6; ++stages) {
+        const size_t smem = rotquant_smem_bytes(stages, stage_bytes, W);
+        if (smem > 227 * 1024) break;
+        const int occ = rotquant_occupancy<T>(gps, threads, smem, dev);
+        if (occ < 1) break;
+        const double busy = double(slots) / double(4 * W * gps);
+        const double inflight = double(occ) * stages * stage_bytes;
+        const double score = occ * W * busy + 4.0 * (inflight < 131072.0 ? inflight : 131072.0) / 131072.0 -
+                             0.01 * gps - 0.001 * R;
+        if (score > best_score) {
+          best_score = score;
+          best = {gps, W, R, stages};
+          best_occ = occ;
         }
       }
+    }
   if (dev >= 0 && dev < 16 && G <= 64 && best.gps != 0) {
     cache[dev][G] = best;
     cache_occ[dev][G] = best_occ;
@@ -434,8 +544,28 @@ RqShape rotquant_plan(int K, int dev, int* blocks_per_sm) {
   return best;
 }
 
+// Fills the kernel arguments for a plan; the tensor map for x is built by the
+// caller with the box {128 / sizeof(T), units_per_copy, R}.
 template <typename T>
-cudaError_t launch_rotquant(const T* x, int64_t rows, int64_t K, int8_t* q, float* s, uint64_t wait_limit_ns,
+RqArgs rotquant_args(const RqShape& sh, int64_t rows, int64_t K, int8_t* q, float* s, uint64_t wait_limit_ns) {
+  RqArgs a;
+  a.M = rows;
+  a.K = static_cast<int>(K);
+  a.R = sh.rows;
+  a.items = (rows + sh.rows - 1) / sh.rows;
+  rotquant_copies<T>(a.K, &a.copies, &a.units_per_copy);
+  a.copy_bytes = rotquant_copy_bytes<T>(a.K, sh.rows);
+  a.stage_bytes = uint32_t(a.copies) * a.copy_bytes;
+  a.tx_bytes = uint32_t(a.copies) * uint32_t(sh.rows) * uint32_t(a.units_per_copy) * 128u;
+  a.stages = sh.stages;
+  a.q = q;
+  a.s_out = s;
+  a.wait_limit_ns = wait_limit_ns;
+  return a;
+}
+
+template <typename T>
+cudaError_t launch_rotquant(const CUtensorMap& tmap, const RqShape& sh, int occ, const RqArgs& a,
                             cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -443,30 +573,14 @@ cudaError_t launch_rotquant(const T* x, int64_t rows, int64_t K, int8_t* q, floa
   static int sm_count[16] = {};
   if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
   if (sm_count[dev] == 0) cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
-  int occ = 0;
-  const RqShape sh = rotquant_plan<T>(static_cast<int>(K), dev, &occ);
-  if (sh.gps == 0) return cudaErrorInvalidConfiguration;
-  RqArgs a;
-  a.M = rows;
-  a.K = static_cast<int>(K);
-  a.R = sh.rows;
-  a.items = (rows + sh.rows - 1) / sh.rows;
-  a.stage_bytes = static_cast<uint32_t>(int64_t(sh.rows) * K * int64_t(sizeof(T)));
-  a.stages = sh.stages;
-  a.q = q;
-  a.s_out = s;
-  a.wait_limit_ns = wait_limit_ns;
   const size_t smem = rotquant_smem_bytes(sh.stages, a.stage_bytes, sh.warps);
   const int threads = 32 * (sh.warps + 1);
   const int64_t cap = int64_t(sm_count[dev]) * occ;
   const unsigned grid = static_cast<unsigned>(a.items < cap ? a.items : cap);
-  if (sh.gps == 1) {
-    if (sh.small) rotquant_kernel<T, 1, true><<<grid, threads, smem, stream>>>(x, a);
-    else rotquant_kernel<T, 1, false><<<grid, threads, smem, stream>>>(x, a);
-  } else {
-    if (sh.small) rotquant_kernel<T, 2, true><<<grid, threads, smem, stream>>>(x, a);
-    else rotquant_kernel<T, 2, false><<<grid, threads, smem, stream>>>(x, a);
-  }
+  if (sh.gps == 1)
+    rotquant_kernel<T, 1><<<grid, threads, smem, stream>>>(tmap, a);
+  else
+    rotquant_kernel<T, 2><<<grid, threads, smem, stream>>>(tmap, a);
   return cudaGetLastError();
 }
 
