@@ -265,7 +265,9 @@ h3q_status h3q_get_device_status(cudaStream_t stream);
 void h3q_set_wait_limit_ns(uint64_t ns);
 
 /*
- * Test hook for the bounded-wait path: launches one block that waits on an
+ * Test hook for the bounded-wait path: launches one block whose threads wait,
+ * through both of the library's bounded-wait forms (the one single issuing
+ * threads use and the one the consumers of a shared-memory ring use), on an
  * mbarrier nothing ever arrives on, with the given limit; afterwards
  * h3q_get_device_status returns H3Q_ERR_TIMEOUT. No fault, no hang.
  */

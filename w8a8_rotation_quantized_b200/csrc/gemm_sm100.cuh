@@ -406,14 +406,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 // arrives on; the wait gives up after limit_ns and records the timeout.
 __global__ void stalled_wait_kernel(uint64_t limit_ns) {
   __shared__ uint64_t bar;
-  __shared__ int abort_flag;
+  __shared__ int abort_flag[2];
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
-    abort_flag = 0;
+    abort_flag[0] = 0;
+    abort_flag[1] = 0;
     fence_mbarrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, limit_ns, &abort_flag);
+  // thread 0 through the issuing-thread helper, warp 1 through the ring-consumer
+  // helper, each with its own abort flag so that each runs into its own limit
+  if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, limit_ns, &abort_flag[0]);
+  if (threadIdx.x >= 32) mbar_wait_bounded_lazy(&bar, 0, limit_ns, &abort_flag[1]);
   __syncthreads();
 }
 

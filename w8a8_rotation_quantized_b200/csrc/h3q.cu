@@ -559,7 +559,7 @@ h3q_status h3q_get_device_status(cudaStream_t stream) {
 
 h3q_status h3q_test_stalled_wait(uint64_t limit_ns, cudaStream_t stream) {
   if (limit_ns > 10000000000ull) return H3Q_ERR_INVALID_ARG;  // at most 10 s
-  h3q::stalled_wait_kernel<<<1, 32, 0, stream>>>(limit_ns < 1000 ? 1000 : limit_ns);
+  h3q::stalled_wait_kernel<<<1, 64, 0, stream>>>(limit_ns < 1000 ? 1000 : limit_ns);
   return cudaGetLastError() == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
 }
 

@@ -97,6 +97,32 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// mbar_wait_bounded for waits that many threads make at once (the consumers of
+// a shared-memory ring): no clock reading unless 64 tries fail, the first
+// reading then starting the limit, so a satisfied or short wait costs only the
+// try_wait loop. (Single issuing threads keep mbar_wait_bounded, whose clock
+// reading after the first failed try spaces out their retries; measured faster
+// there.)
+__device__ __forceinline__ bool mbar_wait_bounded_lazy(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                                       volatile int* abort) {
+  uint32_t spins = 0;
+  uint64_t t0 = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++spins & 63u) == 0) {
+      if (abort != nullptr && *abort) return false;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > limit_ns) {
+        atomicOr(&g_status, kStatusTimeout);
+        if (abort != nullptr) *abort = 1;
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -20,7 +20,8 @@
 //   phase B  lane l holds elements 32 j + 4 l + i (j = 0..7, i = 0..3) and
 //            applies the butterflies of bits 5-7.
 // Values are kept as pairs (v[2i], v[2i+1]): bit 0 is one scalar add and one
-// scalar subtract per pair (fused with the bf16 unpacking), every other bit runs
+// scalar subtract per pair (for bf16 the mixed-precision add reads the low
+// element straight from the packed word), every other bit runs
 // on the sm_100 two-wide fp32 add and FMA. The bits are processed in ascending
 // order and every butterfly is one correctly rounded fp32 add or subtract, so
 // each rotated value has the same bits as the pairwise-tree sum of the explicit
@@ -92,8 +93,15 @@ struct LaneLoad<__nv_bfloat16> {
       const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {  // element 2i of a word is its low half
-        const float lo = __uint_as_float(__byte_perm(u[i], 0u, 0x1044)), hi = __uint_as_float(u[i] & 0xFFFF0000u);
-        p[4 * k + i] = make_float2(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
+        // lo + hi and lo - hi, each one rounding: the sm_100 mixed-precision add
+        // takes the bf16 low half as it is and the high half masked to fp32
+        const float hi = __uint_as_float(u[i] & 0xFFFF0000u);
+        float sum, dif;
+        asm("{\n\t.reg .b16 l16, h16;\n\tmov.b32 {l16, h16}, %2;\n\t"
+            "add.rn.f32.bf16 %0, l16, %3;\n\tsub.rn.f32.bf16 %1, l16, %3;\n\t}"
+            : "=f"(sum), "=f"(dif)
+            : "r"(u[i]), "f"(hi));
+        p[4 * k + i] = make_float2(sum, dif);
       }
     }
   }
@@ -257,7 +265,7 @@ struct RqArgs {
   int64_t M;             // rows
   int K;                 // row length (multiple of 256)
   int R;                 // rows per work item
-  int64_t items;         // ceil(M / R)
+  int items;             // ceil(M / R) (M < 2^31)
   int stages;            // shared-memory ring depth
   uint32_t stage_bytes;  // copies * copy_bytes
   uint32_t copy_bytes;   // shared-memory room of one TMA box, its bytes rounded up to 1024
@@ -335,7 +343,7 @@ __global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
-      for (int64_t item = blockIdx.x; item < a.items; item += gridDim.x) {
+      for (int item = blockIdx.x; item < a.items; item += gridDim.x) {
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_limit_ns, abort_flag)) {
           ok = false;
           break;
@@ -344,7 +352,7 @@ __global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
         const uint32_t dst = stage0 + uint32_t(stage) * a.stage_bytes;
         for (int c = 0; c < a.copies; ++c)
           tma_load_3d(dst + uint32_t(c) * a.copy_bytes, &tmap, &full[stage], 0, c * a.units_per_copy,
-                      static_cast<int32_t>(item * a.R), pol);
+                      item * a.R, pol);
         ++issued;
         if (++stage == a.stages) {
           stage = 0;
@@ -385,11 +393,11 @@ __global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
   int stage = 0;
   uint32_t phase = 0;
   int buf = 0, next = kRqMaxRows;  // offsets of buffers it % 3 and (it + 1) % 3
-  for (int64_t item = blockIdx.x; item < a.items; item += gridDim.x) {
-    mbar_wait_bounded(&full[stage], phase, a.wait_limit_ns, abort_flag);  // on expiry: garbage, no hang
+  for (int item = blockIdx.x; item < a.items; item += gridDim.x) {
+    mbar_wait_bounded_lazy(&full[stage], phase, a.wait_limit_ns, abort_flag);  // on expiry: garbage, no hang
     const uint32_t tile = stage0 + uint32_t(stage) * a.stage_bytes;
     if (c < kRqMaxRows) row_amax[next + c] = 0u;
-    const int64_t row0 = item * a.R;
+    const int64_t row0 = int64_t(item) * a.R;
 
     float2 p[GPS][16];
 #pragma unroll
@@ -552,7 +560,7 @@ RqArgs rotquant_args(const RqShape& sh, int64_t rows, int64_t K, int8_t* q, floa
   a.M = rows;
   a.K = static_cast<int>(K);
   a.R = sh.rows;
-  a.items = (rows + sh.rows - 1) / sh.rows;
+  a.items = static_cast<int>((rows + sh.rows - 1) / sh.rows);
   rotquant_copies<T>(a.K, &a.copies, &a.units_per_copy);
   a.copy_bytes = rotquant_copy_bytes<T>(a.K, sh.rows);
   a.stage_bytes = uint32_t(a.copies) * a.copy_bytes;
