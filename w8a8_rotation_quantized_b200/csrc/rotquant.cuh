@@ -84,8 +84,7 @@ template <typename T>
 struct LaneLoad;
 
 template <>
-struct LaneLoad<__nv_bfloat16> {
-  static constexpr int kChunks = 4;  // 8 elements per 16-byte chunk
+struct LaneLoad<__nv_bfloat16> {  // four chunks of 8 elements
   static __device__ __forceinline__ void load(uint32_t a, float2 (&p)[16]) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -108,8 +107,7 @@ struct LaneLoad<__nv_bfloat16> {
 };
 
 template <>
-struct LaneLoad<float> {
-  static constexpr int kChunks = 8;  // 4 elements per 16-byte chunk
+struct LaneLoad<float> {  // eight chunks of 4 elements
   static __device__ __forceinline__ void load(uint32_t a, float2 (&p)[16]) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
