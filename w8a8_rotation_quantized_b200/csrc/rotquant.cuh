@@ -396,6 +396,7 @@ __global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
     const uint32_t tile = stage0 + uint32_t(stage) * a.stage_bytes;
     if (c < kRqMaxRows) row_amax[next + c] = 0u;
     const int64_t row0 = int64_t(item) * a.R;
+    const int rows_here = a.M - row0 < a.R ? static_cast<int>(a.M - row0) : a.R;  // the item's rows inside M
 
     float2 p[GPS][16];
 #pragma unroll
@@ -411,18 +412,17 @@ __global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
       float m = group_lane_absmax(p[t]);
 #pragma unroll
       for (int o = 1; o <= 4; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-      if (l == 0 && act[t] && row0 + rr[t] < a.M) atomicMax(&row_amax[buf + rr[t]], __float_as_uint(m));
+      if (l == 0 && act[t] && rr[t] < rows_here) atomicMax(&row_amax[buf + rr[t]], __float_as_uint(m));
     }
     named_barrier(1, n_cons);
+    if (c < rows_here)  // one thread per row stores its scale s = s16 / 16
+      a.s_out[row0 + c] = __fmul_rn(div127(__uint_as_float(row_amax[buf + c])), 0.0625f);
 #pragma unroll
     for (int t = 0; t < GPS; ++t) {
-      const int64_t row = row0 + rr[t];
-      const float am = __uint_as_float(row_amax[buf + rr[t]]);
-      const float s16 = div127(am);
-      if (l == 0 && gg[t] == 0 && act[t] && row < a.M) a.s_out[row] = __fmul_rn(s16, 0.0625f);
-      if (act[t] && row < a.M) {
+      const float s16 = div127(__uint_as_float(row_amax[buf + rr[t]]));
+      if (act[t] && rr[t] < rows_here) {
         const RowQuot rq = row_quotient(s16);
-        int8_t* out = a.q + row * a.K + 256 * gg[t] + 4 * l;
+        int8_t* out = a.q + (row0 + rr[t]) * a.K + 256 * gg[t] + 4 * l;
         if (rq.f == 1.0f)
           quantize_store<false>(p[t], rq, out);
         else
