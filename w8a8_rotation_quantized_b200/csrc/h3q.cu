@@ -207,14 +207,14 @@ template <typename T>
 h3q_status run_rotquant(const T* x, int64_t rows, int64_t K, int8_t* q, float* s, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return H3Q_ERR_CUDA;
-  int occ = 0;
-  const h3q::RqShape sh = h3q::rotquant_plan<T>(static_cast<int>(K), dev, &occ);
-  if (sh.gps == 0 || occ < 1) return H3Q_ERR_CUDA;
+  int occ = 0, sms = 0;
+  const h3q::RqShape sh = h3q::rotquant_plan<T>(static_cast<int>(K), dev, &occ, &sms);
+  if (sh.gps == 0 || occ < 1 || sms < 1) return H3Q_ERR_CUDA;
   const h3q::RqArgs a = h3q::rotquant_args<T>(sh, rows, K, q, s, g_wait_limit_ns.load());
   CUtensorMap map;
   if (!make_tmap_rows(&map, x, rows, K, static_cast<int>(sizeof(T)), a.units_per_copy, sh.rows))
     return H3Q_ERR_CUDA;
-  return h3q::launch_rotquant<T>(map, sh, occ, a, stream) == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+  return h3q::launch_rotquant<T>(map, sh, occ, sms, a, stream) == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
 }
 
 bool valid_k(int64_t K) { return K >= 256 && K % 256 == 0; }

@@ -48,6 +48,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "ptx_sm100.cuh"
 
 namespace h3q {
@@ -435,7 +437,14 @@ __global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
 }
 
 // ----------------------------------------------------------------------------
-// Host side: shape choice and launch.
+// Host side: shape choice and launch. The per-device host caches below (kernel
+// attributes set, chosen shape and occupancy per row length, SM count) are
+// read and written only under this mutex, which rotquant_plan holds.
+
+inline std::mutex& rotquant_host_mutex() {
+  static std::mutex m;
+  return m;
+}
 
 template <typename T, int GPS>
 cudaError_t rotquant_prepare_attr(int dev) {
@@ -493,11 +502,20 @@ inline uint32_t rotquant_copy_bytes(int K, int R) {
 // (3.5 TB/s); K = 14336: two groups per quarter, 7 warps, one row per item
 // (3.7 TB/s).
 template <typename T>
-RqShape rotquant_plan(int K, int dev, int* blocks_per_sm) {
+RqShape rotquant_plan(int K, int dev, int* blocks_per_sm, int* sms) {
+  std::lock_guard<std::mutex> lock(rotquant_host_mutex());
   static RqShape cache[16][65] = {};
   static int cache_occ[16][65] = {};
+  static int sm_count[16] = {};
+  *blocks_per_sm = 0;
+  *sms = 0;
+  if (dev < 0 || dev >= 16) return RqShape{0, 0, 0, 0};
+  if (sm_count[dev] == 0 &&
+      cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return RqShape{0, 0, 0, 0};
+  *sms = sm_count[dev];
   const int G = K / 256;
-  if (dev >= 0 && dev < 16 && G <= 64 && cache[dev][G].gps != 0) {
+  if (G <= 64 && cache[dev][G].gps != 0) {
     *blocks_per_sm = cache_occ[dev][G];
     return cache[dev][G];
   }
@@ -542,7 +560,7 @@ RqShape rotquant_plan(int K, int dev, int* blocks_per_sm) {
         }
       }
     }
-  if (dev >= 0 && dev < 16 && G <= 64 && best.gps != 0) {
+  if (G <= 64 && best.gps != 0) {
     cache[dev][G] = best;
     cache_occ[dev][G] = best_occ;
   }
@@ -570,18 +588,13 @@ RqArgs rotquant_args(const RqShape& sh, int64_t rows, int64_t K, int8_t* q, floa
   return a;
 }
 
+// Launches a plan: a persistent grid of min(items, SMs x blocks per SM) blocks.
 template <typename T>
-cudaError_t launch_rotquant(const CUtensorMap& tmap, const RqShape& sh, int occ, const RqArgs& a,
+cudaError_t launch_rotquant(const CUtensorMap& tmap, const RqShape& sh, int occ, int sms, const RqArgs& a,
                             cudaStream_t stream) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  static int sm_count[16] = {};
-  if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
-  if (sm_count[dev] == 0) cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
   const size_t smem = rotquant_smem_bytes(sh.stages, a.stage_bytes, sh.warps);
   const int threads = 32 * (sh.warps + 1);
-  const int64_t cap = int64_t(sm_count[dev]) * occ;
+  const int64_t cap = int64_t(sms) * occ;
   const unsigned grid = static_cast<unsigned>(a.items < cap ? a.items : cap);
   if (sh.gps == 1)
     rotquant_kernel<T, 1><<<grid, threads, smem, stream>>>(tmap, a);
