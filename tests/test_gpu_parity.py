@@ -51,7 +51,10 @@ def assert_bf16_close(got, want, where):
 @pytest.mark.parametrize("M,K", [(1, 256), (7, 512), (64, 512), (129, 768), (300, 5376), (33, 14336),
                                  (5, 16384), (130, 1280), (17, 256),
                                  # more rows than SMs, so blocks cycle their ring and the row buffers
-                                 (300, 14336), (20, 7168), (1000, 5376), (601, 10752)])
+                                 (300, 14336), (20, 7168), (1000, 5376), (601, 10752),
+                                 # K = 5376 takes two rows per work item: an odd M leaves the last
+                                 # item one real row (the other reads as zeros and is not written)
+                                 (301, 5376), (1, 5376)])
 def test_rotate_quant_bitexact(h3q, cuda_device, M, K):
     bits, to_dev = _u(cuda_device)
     f = synth.column_factors(K, synth.outlier_columns(0, 4, K, max(1, K // 100)), 50.0)
