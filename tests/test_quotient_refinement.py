@@ -49,3 +49,16 @@ def test_candidate_code_with_residual_check_equals_rounded_ieee_quotient(tmp_pat
     assert cases == 40_000_000
     assert bad == 0, out.stderr
     assert fallbacks >= cases // 3
+
+
+def test_code_check_catches_a_loose_residual_bound(tmp_path):
+    """The same check with the bound at exactly s/2 (no margin for the rounding of y/s)
+    must report mismatches: the exact half-integer quotients then pass the residual test
+    with the wrong candidate."""
+    exe = tmp_path / "code_check_loose"
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-DBOUND=0.5f", "-o", str(exe),
+                           os.path.join(HERE, "csrc", "code_check.c"), "-lm"])
+    out = subprocess.run([str(exe), "200", "2000"], capture_output=True, text=True, check=True)
+    bad, cases, _ = map(int, out.stdout.split())
+    assert cases == 400_000
+    assert bad > 0
