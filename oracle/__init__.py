@@ -50,6 +50,8 @@ def _load():
             "orc_epilogue": (None, [P, P, P, P, I64, I64, P, P]),
             "orc_exp_f32": (F, [F]),
             "orc_silu_f32": (F, [F]),
+            "orc_exp_f32_array": (None, [P, I64, P]),
+            "orc_silu_f32_array": (None, [P, I64, P]),
             "orc_swiglu": (None, [P, I64, I64, P, P]),
             "orc_linear": (I64, [P, I64, I64, P, P, I64, P, ctypes.c_int, P, P, P, P, P]),
             "orc_ffn": (I64, [P, I64, I64, P, P, P, I64, P, P, P, P, P, P, P]),
@@ -188,6 +190,20 @@ def exp_f32(t: float) -> float:
 
 def silu_f32(g: float) -> float:
     return float(_load().orc_silu_f32(float(g)))
+
+
+def exp_f32_array(t: np.ndarray) -> np.ndarray:
+    t = np.ascontiguousarray(t, dtype=np.float32)
+    out = np.empty_like(t)
+    _load().orc_exp_f32_array(t.ctypes.data, t.size, out.ctypes.data)
+    return out
+
+
+def silu_f32_array(g: np.ndarray) -> np.ndarray:
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    out = np.empty_like(g)
+    _load().orc_silu_f32_array(g.ctypes.data, g.size, out.ctypes.data)
+    return out
 
 
 def swiglu(v):

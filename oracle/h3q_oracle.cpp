@@ -29,7 +29,8 @@
 // one scale per token over the whole row; epilogue order
 // ((float)acc * sx) * sw + bias without fused multiply-add; SwiGLU takes the
 // first half of the fc1 outputs as gate and the second half as up; e^-g is
-// evaluated by Cody-Waite reduction and a degree-7 Taylor polynomial in fp32;
+// evaluated by Cody-Waite reduction and a degree-7 Taylor polynomial in fp32,
+// with the power of two moved onto the numerator where e^-g >= 2^64;
 // the LoRA delta B A_rot is a fused multiply-add chain over the rank index in
 // ascending order, scaled by alpha and added to q * s as two rounded products
 // and one rounded add.
@@ -215,16 +216,16 @@ void orc_epilogue(const int32_t* acc, const float* sx, const float* sw, const ui
 }
 
 // ---------------------------------------------------------------------------
-// Step 8: SwiGLU, h = silu(g) * u with silu(g) = g / (1 + e^-g).
-// e^t is evaluated in fp32 by Cody-Waite reduction t = n ln2 + r (the two-part
-// ln2 of fdlibm's expf: 0x3f317200 and 0x35bfbe8e), then e^r by the degree-7
-// Taylor polynomial in Horner form with fused multiply-adds, then scaled by 2^n.
-// For t > 88 the value is +inf (silu -> -0); for t < -20, 1 + e^t rounds to 1
-// in fp32 whatever e^t is, so e^t is taken as 0.
+// Step 8: SwiGLU, h = silu(g) * u with silu(g) = g / (1 + e^-g) (h3-rs README,
+// "Speed", "What makes it fast": SwiGLU in fc1's epilogue).
+// e^t is evaluated in fp32 as p * 2^n: Cody-Waite reduction t = n ln2 + r with
+// n = rne(t log2 e) and the two-part ln2 of fdlibm's expf (0x3f317200 and
+// 0x35bfbe8e), then p = e^r by the degree-7 Taylor polynomial in Horner form
+// with fused multiply-adds. e^t itself is p scaled by 2^n (ldexp: exact, +inf
+// only where the scaled value overflows fp32, i.e. t above ln(FLT_MAX) ~ 88.72).
+// For t < -20, 1 + e^t rounds to 1 in fp32 whatever e^t is, so e^t is taken as 0.
 // ---------------------------------------------------------------------------
-float orc_exp_f32(float t) {
-  if (t > 88.0f) return INFINITY;
-  if (t < -20.0f) return 0.0f;
+static void exp_parts(float t, float* p_out, int* n_out) {
   const float n = std::nearbyint(t * 1.44269502f);   // log2(e) rounded to fp32
   float r = std::fma(n, -0.693145751953125f, t);     // ln2 high part (0x3f317200)
   r = std::fma(n, -1.42860677e-06f, r);              // ln2 low part  (0x35bfbe8e)
@@ -236,10 +237,46 @@ float orc_exp_f32(float t) {
   p = std::fma(p, r, 0.5f);
   p = std::fma(p, r, 1.0f);
   p = std::fma(p, r, 1.0f);
-  return std::ldexp(p, int(n));
+  *p_out = p;
+  *n_out = int(n);
 }
 
-float orc_silu_f32(float g) { return g / (1.0f + orc_exp_f32(-g)); }
+float orc_exp_f32(float t) {
+  if (t < -20.0f) return 0.0f;
+  if (t > 89.0f) return INFINITY;                    // e^t > FLT_MAX for t > 88.73
+  float p;
+  int n;
+  exp_parts(t, &p, &n);
+  return std::ldexp(p, n);
+}
+
+// silu(g) = RN(g / RN(1 + e^-g)). Where e^-g is at least 2^64 (g below about
+// -44.4), 1 + e^-g rounds to e^-g = p * 2^n, and the quotient g / (p * 2^n) is
+// formed as (g * 2^(64-n)) / (p * 2^64): both operands are exact, so this is the
+// same correctly rounded quotient, and it stays right where e^-g itself
+// overflows fp32 (g < -88.72) down to where silu underflows. For g < -120,
+// |silu(g)| < 2^-160 and the result is -0.
+float orc_silu_f32(float g) {
+  const float t = -g;
+  if (t < -20.0f) return g;
+  if (t > 120.0f) return -0.0f;
+  float p;
+  int n;
+  exp_parts(t, &p, &n);
+  if (n <= 64) return g / (1.0f + std::ldexp(p, n));
+  return std::ldexp(g, 64 - n) / std::ldexp(p, 64);
+}
+
+// Element-wise forms of the two functions above, for checking them over many arguments.
+void orc_exp_f32_array(const float* t, int64_t n, float* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_exp_f32(t[i]);
+}
+
+void orc_silu_f32_array(const float* g, int64_t n, float* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_silu_f32(g[i]);
+}
 
 // v [M, 2F] (epilogue values of the fc1 rows: gate = [0,F), up = [F,2F)).
 void orc_swiglu(const float* v, int64_t M, int64_t F, float* h, uint16_t* out) {

@@ -202,6 +202,34 @@ def test_linear_swiglu_bitexact(h3q, cuda_device, M, K, F, with_bias):
     assert np.array_equal(got, want), f"{(got != want).sum()} of {got.size} differ (within 1 ulp)"
 
 
+def test_swiglu_gate_values_past_fp32_exp_overflow(h3q, cuda_device):
+    """Gate values over [-400, 400]: silu's e^-g runs past 2^64 (g < -44.4, the quotient
+    taken with the power of two on the numerator), past fp32 overflow (g < -88.72, silu still
+    a nonzero value near g e^g) and past silu's own underflow (g < -104). Bit-exact."""
+    dev = cuda_device
+    M, K, F = 128, 256, 128
+    rng = np.random.default_rng(11)
+    xq_h = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
+    wq_h = rng.integers(-127, 128, size=(2 * F, K), dtype=np.int8)
+    acc = oracle.gemm_s32(xq_h, wq_h)
+    sw_h = np.full(2 * F, 1.0 / float(np.abs(acc).max()), dtype=np.float32)
+    sx_h = np.linspace(1.0, 400.0, M, dtype=np.float32)
+    sw_h[F:] = sw_h[F:] * np.float32(1e30)         # up values large, so h = silu(g) u stays visible
+    v, _ = oracle.epilogue(acc, sx_h, sw_h)
+    g = v[:, :F]
+    assert (g < -120).any() and ((g < -88.8) & (g > -103)).any() and ((g < -44.5) & (g > -88)).any()
+    _, want = oracle.swiglu(v)
+    y = torch.empty((M, F), dtype=torch.bfloat16, device=dev)
+    h3q.h3q_linear_w8a8(torch.from_numpy(xq_h).to(dev), torch.from_numpy(sx_h).to(dev),
+                        torch.from_numpy(wq_h).to(dev), torch.from_numpy(sw_h).to(dev), y,
+                        epilogue=h3q.H3Q_EPI_SWIGLU)
+    torch.cuda.synchronize()
+    got = _u(dev)[0](y)
+    deep = (g < -88.8) & (g > -100)
+    assert np.all(synth.bf16_bits_to_fp32(want)[deep] != 0.0)
+    assert np.array_equal(got, want), f"{(got != want).sum()} of {got.size} differ"
+
+
 # ---------------------------------------------------------------- FFN
 @pytest.mark.parametrize("M,K,F,with_bias", [(70, 512, 768, False), (64, 512, 256, True), (129, 256, 512, True)])
 def test_ffn_bitexact(h3q, cuda_device, M, K, F, with_bias):

@@ -7,6 +7,8 @@ step (a dropped term, a wrong sign or index, a transposed operand, a swapped
 gate/up) fails at least one of them.
 """
 import math
+import os
+import subprocess
 
 import numpy as np
 import pytest
@@ -237,18 +239,65 @@ def test_bf16_rounding_matches_torch():
 
 # --------------------------------------------------------------------- SwiGLU
 def test_exp_and_silu_against_math():
-    ts = np.linspace(-19.9, 30.0, 4001, dtype=np.float32)
+    ts = np.linspace(-19.9, 88.7, 4001, dtype=np.float32)
     for t in ts:
         e = oracle.exp_f32(float(t))
         ref = math.exp(float(t))
         assert abs(e - ref) <= 2 * np.spacing(np.float32(ref)), (t, e, ref)
-    for g in np.linspace(-20, 20, 2001, dtype=np.float32):
+    for g in np.linspace(-100, 100, 2001, dtype=np.float32):
         s = oracle.silu_f32(float(g))
         ref = float(g) / (1.0 + math.exp(-float(g)))
-        assert abs(s - ref) <= 4 * np.spacing(np.float32(abs(ref))) + 1e-45, (g, s, ref)
+        assert abs(s - ref) <= 4 * np.spacing(np.float32(abs(ref))) + 2.0 ** -149, (g, s, ref)
     assert oracle.silu_f32(0.0) == 0.0
     assert oracle.silu_f32(30.0) == 30.0
-    assert oracle.silu_f32(-100.0) == 0.0
+    assert oracle.silu_f32(-130.0) == 0.0 and math.copysign(1.0, oracle.silu_f32(-130.0)) == -1.0
+
+
+def test_exp_finite_up_to_fp32_overflow():
+    """e^t is finite for every fp32 t whose true exponential is at most FLT_MAX (ln FLT_MAX
+    is about 88.7228) and +inf above; silu(g) for g just below -88 (where e^-g is finite
+    but above 2^127) and below -88.72 (where it overflows) is a nonzero value near g e^g."""
+    fmax = float(np.finfo(np.float32).max)
+    t = np.float32(88.0)
+    while math.exp(float(np.nextafter(t, np.float32(np.inf)))) <= fmax:
+        t = np.nextafter(t, np.float32(np.inf))
+    assert math.exp(float(t)) <= fmax < math.exp(float(np.nextafter(t, np.float32(np.inf))))
+    assert math.isfinite(oracle.exp_f32(float(t)))
+    assert abs(oracle.exp_f32(float(t)) - math.exp(float(t))) <= 2 * np.spacing(np.float32(fmax))
+    assert math.isfinite(oracle.exp_f32(88.3)) and oracle.exp_f32(89.5) == math.inf
+    for g in (-88.3, -88.9, -95.0):
+        g32 = float(np.float32(g))
+        s = oracle.silu_f32(g32)
+        ref = g32 / (1.0 + math.exp(-g32))
+        assert s < 0.0 and abs(s - ref) <= 4 * np.spacing(np.float32(abs(ref))) + 2.0 ** -149, (g, s, ref)
+    assert abs(oracle.silu_f32(-88.3)) >= np.finfo(np.float32).tiny          # a normal number
+
+
+def _exp_silu_check(tmp_path):
+    exe = tmp_path / "exp_silu_check"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-o", str(exe),
+                           os.path.join(os.path.dirname(__file__), "csrc", "exp_silu_check.c"), "-lm", "-ldl"])
+
+    def run(*args):
+        out = subprocess.run([str(exe), oracle.build(), *map(str, args)], capture_output=True, text=True,
+                             check=True)
+        checked, bad, worst_milli_ulp = map(int, out.stdout.split())
+        return checked, bad, worst_milli_ulp / 1000.0
+    return run
+
+
+def test_exp_and_silu_over_every_float_against_libm(tmp_path):
+    """Against the C library's double exp, over fp32 arguments: e^t on [-20, 89] within 2 ulps
+    (+inf or FLT_MAX where the true value is above FLT_MAX), silu on [-100, 100] within 4 ulps.
+    Every float in the windows where the cut-offs sit ([87.5, 89] for e^t; [-100, -80] and
+    [-21, -19] for silu, [-20, -19] for e^t, below which it is taken as 0); elsewhere every 13th bit pattern, or every float
+    with H3Q_FULL_EXP_SWEEP=1 (about a minute on 8 cores)."""
+    run = _exp_silu_check(tmp_path)
+    stride = 1 if os.environ.get("H3Q_FULL_EXP_SWEEP") == "1" else 13
+    for args in (("exp", stride), ("exp", 1, 87.5, 89.0), ("exp", 1, -20.0, -19.0),
+                 ("silu", stride), ("silu", 1, -100.0, -80.0), ("silu", 1, -21.0, -19.0)):
+        checked, bad, worst = run(*args)
+        assert checked > 100_000 and bad == 0, (args, checked, bad, worst)
 
 
 def test_swiglu_gate_is_first_half():

@@ -95,13 +95,19 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmParams& p, int& 
   nb = r / gm;
 }
 
-// e^t in fp32: Cody-Waite reduction t = n ln2 + r with fdlibm's two-part ln2
-// (0x3f317200, 0x35bfbe8e), e^r by the degree-7 Taylor polynomial in Horner form
-// with fused multiply-adds, then an exact scale by 2^n. t > 88 gives +inf; for
-// t < -20, 1 + e^t is 1 in fp32, so e^t is taken as 0.
-__device__ __forceinline__ float exp_f32(float t) {
-  if (t > 88.0f) return __int_as_float(0x7F800000);
-  if (t < -20.0f) return 0.0f;
+// silu(g) = g / (1 + e^-g) in fp32 (SwiGLU, h3-rs README, "What makes it fast").
+// e^t = p * 2^n: Cody-Waite reduction t = n ln2 + r with n = rne(t log2 e) and
+// fdlibm's two-part ln2 (0x3f317200, 0x35bfbe8e), p = e^r by the degree-7 Taylor
+// polynomial in Horner form with fused multiply-adds. For t < -20, 1 + e^t is 1
+// in fp32 (silu(g) = g). For n <= 64 the quotient is g / (1 + p 2^n), with 2^n
+// applied by one exact multiply. For n > 64, 1 + e^t rounds to p 2^n, and the
+// quotient is formed as (g 2^(64-n)) / (p 2^64): both operands exact, so it is
+// the same correctly rounded quotient, and it stays right where e^t overflows
+// fp32 (g < -88.72) down to where silu underflows. g < -120 gives -0.
+__device__ __forceinline__ float silu_f32(float g) {
+  const float t = -g;
+  if (t < -20.0f) return g;
+  if (t > 120.0f) return -0.0f;
   // n = rne(t log2 e): adding 1.5 * 2^23 rounds to an integer (ties to even) and
   // leaves it in the low mantissa bits
   const float nm = __fadd_rn(__fmul_rn(t, 1.44269502f), 12582912.0f);
@@ -117,10 +123,10 @@ __device__ __forceinline__ float exp_f32(float t) {
   p = __fmaf_rn(p, r, 0.5f);
   p = __fmaf_rn(p, r, 1.0f);
   p = __fmaf_rn(p, r, 1.0f);
-  return __fmul_rn(p, __int_as_float((ni + 127) << 23));
+  if (__builtin_expect(ni > 64, 0))
+    return __fdiv_rn(__fmul_rn(g, __int_as_float((191 - ni) << 23)), __fmul_rn(p, 18446744073709551616.0f));
+  return __fdiv_rn(g, __fadd_rn(1.0f, __fmul_rn(p, __int_as_float((ni + 127) << 23))));
 }
-
-__device__ __forceinline__ float silu_f32(float g) { return __fdiv_rn(g, __fadd_rn(1.0f, exp_f32(-g))); }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
