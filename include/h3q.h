@@ -130,6 +130,8 @@ h3q_status h3q_ffn(const void* x_bf16, int64_t M, int64_t K,
  *   larger batch into chunks).
  *   The first call on each device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
+ *   After cudaDeviceReset the device has a new context and the next call
+ *   looks the address up again: make that call outside stream capture too.
  *   All calls share the one array and it keeps the last call's contents:
  *   calls that may overlap on the GPU (different streams without ordering
  *   between them, or different host threads) race on it and must be

@@ -151,3 +151,20 @@ def test_attention_rejects():
         args[i] = bad
         assert f(*args) == INV, (i, bad)
     assert f(None, None, None, 0, 2, 256, None, 256, None, 0, None) == h3q.H3Q_OK
+
+
+def test_binding_rejects_host_tensors_and_wrong_dtypes():
+    """The Python binding checks each operand's dtype, device, shape and layout before it
+    builds a pointer: a tensor the kernels would index past its end never reaches them."""
+    torch = pytest.importorskip("torch")
+    x = torch.zeros((4, 256), dtype=torch.bfloat16)
+    xq = torch.zeros((4, 256), dtype=torch.int8)
+    sx = torch.zeros(4, dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        h3q.h3q_rotate_quant(x, xq, sx)
+    with pytest.raises(ValueError, match="must be torch.bfloat16"):
+        h3q.h3q_rotate_quant(x.float(), xq, sx)
+    with pytest.raises(ValueError, match="must be torch.int8"):
+        h3q.h3q_gemm_s32(x, xq, sx)
+    with pytest.raises(ValueError, match="is required"):
+        h3q.h3q_linear_w8a8(None, sx, xq, sx, x)

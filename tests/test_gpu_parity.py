@@ -288,3 +288,35 @@ def test_runs_on_a_side_stream(h3q, cuda_device):
     s.synchronize()
     oq, _ = oracle.rotate_quant_bf16(x_h)
     assert np.array_equal(xq.cpu().numpy(), oq)
+
+
+def test_binding_rejects_wrong_shapes_and_layouts(h3q, cuda_device):
+    """Operands of the wrong shape, a transposed or strided view, or on another device are
+    refused by the binding before any pointer reaches the library."""
+    dev = cuda_device
+    M, K, N, F = 8, 256, 16, 512
+    x = torch.zeros((M, K), dtype=torch.bfloat16, device=dev)
+    xq = torch.zeros((M, K), dtype=torch.int8, device=dev)
+    sx = torch.zeros(M, dtype=torch.float32, device=dev)
+    wq = torch.zeros((N, K), dtype=torch.int8, device=dev)
+    sw = torch.zeros(N, dtype=torch.float32, device=dev)
+    with pytest.raises(ValueError, match="shape"):
+        h3q.h3q_linear_w8a8(xq, sx, wq, sw, torch.zeros((M, N + 8), dtype=torch.bfloat16, device=dev))
+    with pytest.raises(ValueError, match="shape"):
+        h3q.h3q_linear_w8a8(xq, sx, wq, sw, torch.zeros((M, N), dtype=torch.bfloat16, device=dev),
+                            epilogue=h3q.H3Q_EPI_SWIGLU)
+    with pytest.raises(ValueError, match="contiguous"):
+        h3q.h3q_rotate_quant(torch.zeros((K, M), dtype=torch.bfloat16, device=dev).t(), xq, sx)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        h3q.h3q_rotate_quant(x, xq, sx.cpu())
+    w_gu = torch.zeros((2 * F, K), dtype=torch.int8, device=dev)
+    s_gu = torch.zeros(2 * F, dtype=torch.float32, device=dev)
+    w_down_t = torch.zeros((F, K), dtype=torch.int8, device=dev)     # [F, K] instead of [K, F]
+    s_down = torch.zeros(K, dtype=torch.float32, device=dev)
+    ws = torch.empty(h3q.h3q_ffn_workspace_size(M, K, F), dtype=torch.uint8, device=dev)
+    y = torch.zeros((M, K), dtype=torch.bfloat16, device=dev)
+    with pytest.raises(ValueError, match="w_down"):
+        h3q.h3q_ffn(x, w_gu, s_gu, w_down_t, s_down, y, ws)
+    with pytest.raises(ValueError, match="s_down"):
+        h3q.h3q_ffn(x, w_gu, s_gu, torch.zeros((K, F), dtype=torch.int8, device=dev), s_down[:8], y, ws)
+    assert h3q.h3q_get_device_status() == h3q.H3Q_OK

@@ -10,6 +10,8 @@
 #include <cmath>
 #include <atomic>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "h3q.h"
 #include "gemm_sm100.cuh"
@@ -39,6 +41,24 @@ constexpr int kGemmPolicyA = H3Q_GEMM_POLICY_A;
 constexpr int kGemmPolicyB = H3Q_GEMM_POLICY_B;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Kernel attributes belong to the context of the device that is current when
+// they are set, so a process that drives several GPUs sets them once per
+// (kernel, device). The record of what was set is read and written under one
+// mutex; a failed set is not recorded and is retried on the next call.
+std::mutex g_attr_mu;
+std::set<std::pair<const void*, int>> g_attr_done;
+
+cudaError_t ensure_smem_attr(const void* kernel, int smem_bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  if (g_attr_done.count({kernel, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e == cudaSuccess) g_attr_done.insert({kernel, dev});
+  return e;
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -84,13 +104,9 @@ h3q_status launch_gemm(const int8_t* a, const int8_t* b, int64_t M, int64_t K, i
                        const float* sx, const float* sw, const void* bias, void* out, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!make_tmap_i8(&ta, a, M, K) || !make_tmap_i8(&tb, b, b_rows, K)) return H3Q_ERR_CUDA;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(h3q::gemm_i8_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(h3q::kGemmSmem));
-  });
-  if (attr_err != cudaSuccess) return H3Q_ERR_CUDA;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(h3q::gemm_i8_kernel<EPI>),
+                       static_cast<int>(h3q::kGemmSmem)) != cudaSuccess)
+    return H3Q_ERR_CUDA;
   GemmParams p{};
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N_out);
@@ -142,13 +158,9 @@ h3q_status launch_gemm_fp4(const uint8_t* a, const uint8_t* a_sf, const float* a
   if (!make_tmap_i8(&ta, a, M, K / 2) || !make_tmap_i8(&tb, b, b_rows, K / 2) ||
       !make_tmap_sf(&tsa, a_sf, h3q::nvfp4_sf_bytes(M, K)) || !make_tmap_sf(&tsb, b_sf, h3q::nvfp4_sf_bytes(b_rows, K)))
     return H3Q_ERR_CUDA;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(h3q::gemm_fp4_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(h3q::kF4Smem));
-  });
-  if (attr_err != cudaSuccess) return H3Q_ERR_CUDA;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(h3q::gemm_fp4_kernel<EPI>),
+                       static_cast<int>(h3q::kF4Smem)) != cudaSuccess)
+    return H3Q_ERR_CUDA;
   h3q::Fp4Params p{};
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N_out);
@@ -239,20 +251,53 @@ FfnLayout ffn_layout(int64_t M, int64_t K, int64_t F) {
 
 // Scratch for h3q_ffn_static_scratch: a fixed device array, so that call needs
 // no allocation. In host code this name only stands for the array; its device
-// address comes from cudaGetSymbolAddress, once per device.
+// address comes from cudaGetSymbolAddress, looked up with the device current.
 static __device__ __align__(256) unsigned char g_static_scratch[H3Q_STATIC_SCRATCH_BYTES];
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// The current context's ID, unique among all contexts the process creates, so a
+// context re-created after cudaDeviceReset never matches an older one. False if
+// no context is current or the driver lacks the call.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// The array's device address on `device` (the current device), cached per device
+// together with the ID of the context it was looked up in; a new context on that
+// device (after a device reset) looks it up again. Without context IDs from the
+// driver, every call looks it up.
 void* static_scratch_address(int device) {
   static std::mutex mu;
   static void* addr[64] = {};
+  static unsigned long long ctx_id[64] = {};
   if (device < 0 || device >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[device] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+  unsigned long long id = 0;
+  if (addr[device] != nullptr && current_context_id(&id) && id == ctx_id[device]) return addr[device];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+  if (current_context_id(&id)) {  // read after the lookup, which made the device's context current
     addr[device] = p;
+    ctx_id[device] = id;
   }
-  return addr[device];
+  return p;
 }
 
 }  // namespace
@@ -462,18 +507,18 @@ h3q_status h3q_attention_int8(const void* q, const void* k, const void* v, int64
   if (!make_tmap_i8(&tq, qq, H * S, 128) || !make_tmap_i8(&tk, kq, H * S, 128) ||
       !make_tmap_bf16(&tv, vt, H * 128, S))
     return H3Q_ERR_CUDA;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(h3q::attn_kernel), static_cast<int>(h3q::kAttSmem)) !=
+      cudaSuccess)
+    return H3Q_ERR_CUDA;
+  // the kernel's register split assumes this many registers per thread at launch
+  // (a property of the compiled kernel, the same on every device)
+  static std::once_flag regs_once;
   static bool regs_ok = false;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(h3q::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(h3q::kAttSmem));
+  std::call_once(regs_once, [] {
     cudaFuncAttributes fa{};
-    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, h3q::attn_kernel);
-    // the kernel's register split assumes this many registers per thread at launch
-    regs_ok = attr_err == cudaSuccess && fa.numRegs >= static_cast<int>(h3q::kAttRegsLaunch);
+    regs_ok = cudaFuncGetAttributes(&fa, h3q::attn_kernel) == cudaSuccess &&
+              fa.numRegs >= static_cast<int>(h3q::kAttRegsLaunch);
   });
-  if (attr_err != cudaSuccess) return H3Q_ERR_CUDA;
   if (!regs_ok) return H3Q_ERR_UNSUPPORTED;
   h3q::AttParams p{};
   p.S = static_cast<int>(S);
