@@ -36,7 +36,11 @@ std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 #ifndef H3Q_GEMM_POLICY_B
 #define H3Q_GEMM_POLICY_B 1
 #endif
+#ifndef H3Q_GEMM_RASTER
+#define H3Q_GEMM_RASTER 0
+#endif
 constexpr int kGemmGroupRows = H3Q_GEMM_GROUP_ROWS;
+constexpr int kGemmRaster = H3Q_GEMM_RASTER;
 constexpr int kGemmPolicyA = H3Q_GEMM_POLICY_A;
 constexpr int kGemmPolicyB = H3Q_GEMM_POLICY_B;
 
@@ -119,7 +123,7 @@ h3q_status launch_gemm(const int8_t* a, const int8_t* b, int64_t M, int64_t K, i
   // Tile order: groups of kGemmGroupRows pair-row blocks (the group's A tiles are
   // reused by every N block from L2, each B tile is read once per group); both
   // operands are loaded with an evict-last L2 policy.
-  p.raster = 0;
+  p.raster = kGemmRaster;
   p.group_m = kGemmGroupRows < p.num_m ? kGemmGroupRows : p.num_m;
   p.pol_a = kGemmPolicyA;
   p.pol_b = kGemmPolicyB;
