@@ -15,8 +15,9 @@
 //            read from the swizzled stage, so the 8 lanes of a quarter hit 8
 //            different bank quads;
 //   transpose through a per-quarter fp32 scratch of 8 rows with a 144-byte pitch
-//            (each row shifted by one bank quad), written and read in 16-byte
-//            pieces without bank conflicts;
+//            (each row shifted by one bank quad), written in 8-byte pairs (in
+//            odd quarters with the two pairs of each 16-byte slot swapped) and
+//            read in 16-byte pieces, without bank conflicts;
 //   phase B  lane l holds elements 32 j + 4 l + i (j = 0..7, i = 0..3) and
 //            applies the butterflies of bits 5-7.
 // Values are kept as pairs (v[2i], v[2i+1]): bit 0 is one scalar add and one
@@ -147,17 +148,29 @@ __device__ __forceinline__ void butterflies(float2 (&p)[N]) {
 }
 
 // Rotates one group whose lane values (after the bit-0 butterfly, as loaded by
-// LaneLoad) are in p; `scr` is the quarter's scratch and `l` the lane within the
-// quarter. On return p[2j + h] = (y16[32 j + 4 l + 2h], y16[32 j + 4 l + 2h + 1]).
-__device__ __forceinline__ void rotate_group(float* scr, int l, float2 (&p)[16]) {
+// LaneLoad) are in p; `scr` is the quarter's scratch, `l` the lane within the
+// quarter and `odd` the quarter's parity. Phase A's pairs go to the scratch as
+// 8-byte stores, each pair from its own aligned register pair (a 16-byte store
+// would need two pairs moved into one aligned quad first). In an odd quarter pair
+// k goes to slot k ^ 1: the two quarters of a half-warp then write disjoint bank
+// sets (slots 2k, 2k+1 mod 4 against 2k+2, 2k+3 mod 4 words), so each 8-byte store
+// of the warp takes the minimum two wavefronts. Phase B reads 16 bytes per row;
+// in an odd quarter the two halves of each read are swapped, which the
+// butterflies of bits 5-7 (across rows) do not see and the code packing undoes.
+// On return p[2j + h] = (y16[32 j + 4 l + 2 (h ^ odd)], y16[32 j + 4 l + 2 (h ^ odd) + 1]).
+__device__ __forceinline__ void rotate_group(float* scr, int l, int odd, float2 (&p)[16]) {
   butterflies<16, 0, 4, 1>(p);  // index bits 1-4
   float* row = scr + (kRqRowPitch / 4) * l;
+  float* even_base = row + 2 * odd;  // pair k (k even) at slot k + odd
+  float* odd_base = row - 2 * odd;   // pair k (k odd) at slot k - odd
 #pragma unroll
-  for (int k = 0; k < 8; ++k)  // elements 4k .. 4k+3 of row l
-    *reinterpret_cast<float4*>(row + 4 * k) = make_float4(p[2 * k].x, p[2 * k].y, p[2 * k + 1].x, p[2 * k + 1].y);
+  for (int k = 0; k < 16; k += 2) {
+    *reinterpret_cast<float2*>(even_base + 2 * k) = p[k];
+    *reinterpret_cast<float2*>(odd_base + 2 * k + 2) = p[k + 1];
+  }
   __syncwarp();
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {  // elements 4l .. 4l+3 of row j
+  for (int j = 0; j < 8; ++j) {  // slots 2l, 2l+1 of row j
     const float4 c = *reinterpret_cast<const float4*>(scr + (kRqRowPitch / 4) * j + 4 * l);
     p[2 * j] = make_float2(c.x, c.y);
     p[2 * j + 1] = make_float2(c.z, c.w);
@@ -212,7 +225,9 @@ __device__ __forceinline__ RowQuot row_quotient(float s16) {
 }
 
 // int8 codes rne(RN(y16 / s16)) of this lane's 32 values, stored as one 32-bit
-// word per j at out + 32 j (out = the row's codes + 256 g + 4 l).
+// word per j at out + 32 j (out = the row's codes + 256 g + 4 l). `sel` orders the
+// word's two code pairs: 0x5410 when p[2j] holds elements 4l, 4l+1 of row j, 0x1054
+// when it holds 4l+2, 4l+3 (an odd quarter, see rotate_group).
 //
 // Fast path, three fp32 operations per value: the candidate n = rne(y rs) comes
 // from one FMA onto 1.5*2^23 (whose bits then hold n in the low byte), and the
@@ -225,7 +240,8 @@ __device__ __forceinline__ RowQuot row_quotient(float s16) {
 // 2^64 (scale below 2^-100); otherwise f = 1 and the exact rescaling is skipped.
 // An all-zero row has s = 0, rs = 0, t = 0 and residuals 0: codes 0.
 template <bool kRescaled>
-__device__ __forceinline__ void quantize_store(const float2 (&p)[16], const RowQuot& rq, int8_t* out) {
+__device__ __forceinline__ void quantize_store(const float2 (&p)[16], const RowQuot& rq, uint32_t sel,
+                                               int8_t* out) {
   const float2 magic = make_float2(12582912.0f, 12582912.0f), nmagic = make_float2(-12582912.0f, -12582912.0f);
   const float2 f2 = make_float2(rq.f, rq.f), r2 = make_float2(rq.rs, rq.rs), ns2 = make_float2(-rq.sf, -rq.sf);
   const float t = __fmul_rn(rq.sf, 0.4999847412109375f);  // 1/2 - 2^-16
@@ -257,7 +273,7 @@ __device__ __forceinline__ void quantize_store(const float2 (&p)[16], const RowQ
   for (int j = 0; j < 8; ++j) {
     const uint32_t lo = __byte_perm(__float_as_uint(u[2 * j].x), __float_as_uint(u[2 * j].y), 0x0040);
     const uint32_t hi = __byte_perm(__float_as_uint(u[2 * j + 1].x), __float_as_uint(u[2 * j + 1].y), 0x0040);
-    *reinterpret_cast<uint32_t*>(out + 32 * j) = __byte_perm(lo, hi, 0x5410);
+    *reinterpret_cast<uint32_t*>(out + 32 * j) = __byte_perm(lo, hi, sel);
   }
 }
 
@@ -374,6 +390,8 @@ __global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
   const int c = threadIdx.x - 32;
   const int l = c & 7;
   const int qd = c >> 3;
+  const int odd = qd & 1;
+  const uint32_t sel = odd ? 0x1054u : 0x5410u;
   float* scr = scratch_base + size_t(qd) * (kRqScratchBytes / 4);
   int rr[GPS], gg[GPS];
   bool act[GPS];
@@ -410,7 +428,7 @@ __global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
     }
 #pragma unroll
     for (int t = 0; t < GPS; ++t) {
-      rotate_group(scr, l, p[t]);
+      rotate_group(scr, l, odd, p[t]);
       float m = group_lane_absmax(p[t]);
 #pragma unroll
       for (int o = 1; o <= 4; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -426,9 +444,9 @@ __global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
         const RowQuot rq = row_quotient(s16);
         int8_t* out = a.q + (row0 + rr[t]) * a.K + 256 * gg[t] + 4 * l;
         if (rq.f == 1.0f)
-          quantize_store<false>(p[t], rq, out);
+          quantize_store<false>(p[t], rq, sel, out);
         else
-          quantize_store<true>(p[t], rq, out);
+          quantize_store<true>(p[t], rq, sel, out);
       }
     }
     buf = next;
