@@ -54,7 +54,12 @@ def assert_bf16_close(got, want, where):
                                  (300, 14336), (20, 7168), (1000, 5376), (601, 10752),
                                  # K = 5376 takes two rows per work item: an odd M leaves the last
                                  # item one real row (the other reads as zeros and is not written)
-                                 (301, 5376), (1, 5376)])
+                                 (301, 5376), (1, 5376),
+                                 # 8192 rows or more at up to 42 groups run the tensor-memory kernel
+                                 # (values parked in tensor memory, two work items in flight, row
+                                 # maxima in tagged buffers): 3 rows per item at K = 5376, so 8194
+                                 # leaves a last item of one row; K = 10752 takes the searched shape
+                                 (8192, 5376), (8194, 5376), (8195, 10752)])
 def test_rotate_quant_bitexact(h3q, cuda_device, M, K):
     bits, to_dev = _u(cuda_device)
     f = synth.column_factors(K, synth.outlier_columns(0, 4, K, max(1, K // 100)), 50.0)

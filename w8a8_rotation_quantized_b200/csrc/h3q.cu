@@ -219,11 +219,30 @@ bool make_tmap_rows(CUtensorMap* map, const void* base, int64_t rows, int64_t K,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Which rotate+quantize kernel runs: the tensor-memory variant where it measured
+// faster (bf16 rows of up to 42 groups with 8192 rows or more: K = 5376 at 8192 to
+// 32768 rows 4-6% faster, K = 10752 at 16384 rows 10% faster), the register
+// variant otherwise (K = 14336: 5% faster; 4096 rows at K = 5376: 7% faster; fp32
+// weight rows).
+bool rotquant_use_tm(int64_t rows, int64_t K) { return K / 256 <= 42 && rows >= 8192; }
+
 template <typename T>
 h3q_status run_rotquant(const T* x, int64_t rows, int64_t K, int8_t* q, float* s, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return H3Q_ERR_CUDA;
   int occ = 0, sms = 0;
+  if constexpr (sizeof(T) == 2) {
+    if (rotquant_use_tm(rows, K)) {
+      size_t smem = 0;
+      const h3q::RqShape sh = h3q::rotquant_tm_plan<T>(static_cast<int>(K), dev, &occ, &sms, &smem);
+      if (sh.gps == 0 || occ < 1 || sms < 1) return H3Q_ERR_CUDA;
+      const h3q::RqArgs a = h3q::rotquant_args<T>(sh, rows, K, q, s, g_wait_limit_ns.load());
+      CUtensorMap map;
+      if (!make_tmap_rows(&map, x, rows, K, static_cast<int>(sizeof(T)), a.units_per_copy, sh.rows))
+        return H3Q_ERR_CUDA;
+      return h3q::launch_rotquant_tm<T>(map, sh, occ, sms, smem, a, stream) == cudaSuccess ? H3Q_OK : H3Q_ERR_CUDA;
+    }
+  }
   const h3q::RqShape sh = h3q::rotquant_plan<T>(static_cast<int>(K), dev, &occ, &sms);
   if (sh.gps == 0 || occ < 1 || sms < 1) return H3Q_ERR_CUDA;
   const h3q::RqArgs a = h3q::rotquant_args<T>(sh, rows, K, q, s, g_wait_limit_ns.load());

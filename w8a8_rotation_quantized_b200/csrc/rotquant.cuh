@@ -49,6 +49,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "ptx_sm100.cuh"
@@ -122,6 +123,49 @@ struct LaneLoad<float> {  // eight chunks of 4 elements
     }
   }
 };
+
+// The same loads in two steps: the lane's raw 16-byte chunks first (so a stage
+// can be released before any arithmetic), then the unpack with the bit-0
+// butterfly.
+template <typename T>
+struct LaneChunks {
+  static constexpr int kN = 64 / int(sizeof(T)) / 2;  // bf16: 4 chunks, fp32: 8
+  uint4 w[kN];
+  __device__ __forceinline__ void load(uint32_t a) {
+#pragma unroll
+    for (int k = 0; k < kN; ++k) w[k] = lds128(a ^ (16u * k));
+  }
+  __device__ __forceinline__ void unpack(float2 (&p)[16]) const;
+};
+
+template <>
+__device__ __forceinline__ void LaneChunks<__nv_bfloat16>::unpack(float2 (&p)[16]) const {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t u[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float hi = __uint_as_float(u[i] & 0xFFFF0000u);
+      float sum, dif;
+      asm("{\n\t.reg .b16 l16, h16;\n\tmov.b32 {l16, h16}, %2;\n\t"
+          "add.rn.f32.bf16 %0, l16, %3;\n\tsub.rn.f32.bf16 %1, l16, %3;\n\t}"
+          : "=f"(sum), "=f"(dif)
+          : "r"(u[i]), "f"(hi));
+      p[4 * k + i] = make_float2(sum, dif);
+    }
+  }
+}
+
+template <>
+__device__ __forceinline__ void LaneChunks<float>::unpack(float2 (&p)[16]) const {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float v0 = __uint_as_float(w[k].x), v1 = __uint_as_float(w[k].y), v2 = __uint_as_float(w[k].z),
+                v3 = __uint_as_float(w[k].w);
+    p[2 * k] = make_float2(__fadd_rn(v0, v1), __fsub_rn(v0, v1));
+    p[2 * k + 1] = make_float2(__fadd_rn(v2, v3), __fsub_rn(v2, v3));
+  }
+}
 
 // Butterflies over pair indices: for every i with bit b clear,
 // (p[i], p[i + 2^b]) <- (p[i] + p[i + 2^b], p[i] - p[i + 2^b]), bits B0..B1-1 in
@@ -291,11 +335,21 @@ struct RqArgs {
   int8_t* q;
   float* s_out;
   uint64_t wait_limit_ns;
+  uint32_t tmem_cols;    // tensor-memory columns a block allocates (tensor-memory variant)
 };
 
 struct RqShape {
   int gps, warps, rows, stages;  // groups per quarter-warp, consumer warps, rows per item, ring depth
 };
+
+// Tensor-memory columns a block of `warps` consumer warps with `gps` groups per
+// quarter-warp allocates (a power of two, at least 32).
+inline uint32_t rotquant_tm_cols(int warps, int gps) {
+  const uint32_t need = uint32_t((warps + 3) / 4) * 64u * uint32_t(gps);
+  uint32_t c = 32;
+  while (c < need) c <<= 1;
+  return c;
+}
 
 inline size_t rotquant_smem_bytes(int stages, uint32_t stage_bytes, int warps) {
   return 1024 + size_t(stages) * stage_bytes + size_t(4 * warps) * kRqScratchBytes + 2 * sizeof(uint64_t) * stages +
@@ -455,6 +509,209 @@ __global__ void __launch_bounds__(GPS == 1 ? 768 : 512, 1)
 }
 
 // ----------------------------------------------------------------------------
+// Tensor-memory variant. The consumers keep each rotated group in tensor memory
+// (tcgen05.st, 32 columns of the thread's own lane) instead of registers until
+// the row's scale is known, and run two work items at once: in iteration i a
+// thread loads and rotates its groups of item i, posts their maxima and parks
+// the values in tensor-memory slot i % 2, then waits for item i - 1's row maxima
+// (usually complete by then), reads that item's values back (tcgen05.ld) and
+// quantizes them. The row maxima of item i go to buffer i % 4 as 64-bit words
+// (i + 1) << 32 | bits(max) through an atomic max, so a buffer needs no clearing:
+// a newer item's tag exceeds every older value. Completion of an item's maxima
+// is an mbarrier per buffer that each quarter-warp's first lane arrives on after
+// its posts (release), waited on with acquire before the reads. Four buffers
+// suffice: a thread posts item i + 4 only after waiting for item i + 2, which
+// every warp posts only after it has read item i's maxima.
+//
+// Tensor memory: warp w reaches lanes 32 (w % 4) .. 32 (w % 4) + 31; consumer
+// warp w (1..W) takes columns ((w - 1) / 4) 64 GPS .. + 64 GPS of them, two
+// slots of GPS groups of 32 columns.
+constexpr int kRqtMaxRows = 64;
+constexpr int kRqtMaxWarps = 16;
+
+inline size_t rotquant_tm_smem_bytes(int stages, uint32_t stage_bytes, int warps) {
+  return 1024 + size_t(stages) * stage_bytes + size_t(4 * warps) * kRqScratchBytes +
+         sizeof(uint64_t) * (2 * stages + 4) + sizeof(unsigned long long) * 4 * kRqtMaxRows + 16;
+}
+
+template <typename T, int GPS>
+__global__ void __launch_bounds__(32 * (kRqtMaxWarps + 1), 1)
+    rotquant_tm_kernel(const __grid_constant__ CUtensorMap tmap, const RqArgs a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+  uint8_t* smem = smem_raw + pad;  // 1024-byte aligned: stages, then scratch
+  const uint32_t stage0 = raw + pad;
+  const int n_cons = blockDim.x - 32;
+  const int NQ = n_cons >> 3;
+  float* scratch_base = reinterpret_cast<float*>(smem + size_t(a.stages) * a.stage_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(scratch_base) +
+                                               size_t(NQ) * kRqScratchBytes);
+  uint64_t* empty = full + a.stages;
+  uint64_t* rowbar = empty + a.stages;                                                // [4]
+  unsigned long long* rowmax = reinterpret_cast<unsigned long long*>(rowbar + 4);    // [4][kRqtMaxRows]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rowmax + 4 * kRqtMaxRows);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = a.K >> 8;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], n_cons);
+    }
+    for (int b = 0; b < 4; ++b) mbar_init(&rowbar[b], NQ);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  for (int i = threadIdx.x; i < 4 * kRqtMaxRows; i += blockDim.x) rowmax[i] = 0ull;
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, a.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap);
+      const uint64_t pol = policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < a.items; item += gridDim.x) {
+        if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_limit_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], a.tx_bytes);
+        const uint32_t dst = stage0 + uint32_t(stage) * a.stage_bytes;
+        for (int c = 0; c < a.copies; ++c)
+          tma_load_3d(dst + uint32_t(c) * a.copy_bytes, &tmap, &full[stage], 0, c * a.units_per_copy,
+                      item * a.R, pol);
+        ++issued;
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {  // drain this block's own copies still in flight (bounded)
+        for (int s = 0; s < a.stages; ++s) {
+          if (issued <= s) continue;
+          const long last = ((issued - 1 - s) / a.stages) * a.stages + s;
+          mbar_wait_bounded(&full[s], static_cast<uint32_t>((last / a.stages) & 1), a.wait_limit_ns, nullptr);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- consumers
+    const int c = threadIdx.x - 32;
+    const int l = c & 7;
+    const int qd = c >> 3;
+    const int odd = qd & 1;
+    const uint32_t sel = odd ? 0x1054u : 0x5410u;
+    float* scr = scratch_base + size_t(qd) * (kRqScratchBytes / 4);
+    int rr[GPS], gg[GPS];
+    bool act[GPS];
+    uint32_t toff[GPS];
+#pragma unroll
+    for (int t = 0; t < GPS; ++t) {
+      const int i = t * NQ + qd;
+      act[t] = i < a.R * G;
+      rr[t] = act[t] ? i / G : 0;
+      gg[t] = act[t] ? i - rr[t] * G : 0;
+      toff[t] = lane_tile_offset<T>(a, rr[t], gg[t], l);
+    }
+    const uint32_t tm = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
+                        static_cast<uint32_t>(((warp - 1) >> 2) * 64 * GPS);
+    const int n_items = blockIdx.x < a.items ? (a.items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
+
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int it = 0; it <= n_items; ++it) {
+      if (it < n_items) {  // load, rotate, post and park item it
+        const int item = int(blockIdx.x) + it * int(gridDim.x);
+        const int64_t row0 = int64_t(item) * a.R;
+        const int rows_here = a.M - row0 < a.R ? static_cast<int>(a.M - row0) : a.R;
+        const unsigned long long tag = static_cast<unsigned long long>(it + 1) << 32;
+        unsigned long long* rmax = rowmax + (it & 3) * kRqtMaxRows;
+        mbar_wait_bounded_lazy(&full[stage], phase, a.wait_limit_ns, abort_flag);  // on expiry: garbage, no hang
+        const uint32_t tile = stage0 + uint32_t(stage) * a.stage_bytes;
+        LaneChunks<T> raw[GPS];
+#pragma unroll
+        for (int t = 0; t < GPS; ++t) raw[t].load(tile + toff[t]);
+        mbar_arrive(&empty[stage]);  // this thread's reads of the stage are done
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+#pragma unroll
+        for (int t = 0; t < GPS; ++t) {
+          float2 p[16];
+          raw[t].unpack(p);
+          rotate_group(scr, l, odd, p);
+          float m = group_lane_absmax(p);
+#pragma unroll
+          for (int o = 1; o <= 4; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+          if (l == 0 && act[t] && rr[t] < rows_here) atomicMax(&rmax[rr[t]], tag | __float_as_uint(m));
+          uint32_t v[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            v[2 * i] = __float_as_uint(p[i].x);
+            v[2 * i + 1] = __float_as_uint(p[i].y);
+          }
+          tmem_st32(tm + static_cast<uint32_t>(((it & 1) * GPS + t) * 32), v);
+        }
+        __syncwarp();  // every lane of the warp is past its reads of item it - 4's buffer
+        if (l == 0) mbar_arrive(&rowbar[it & 3]);
+      }
+      if (it >= 1) {  // quantize item it - 1
+        const int pit = it - 1;
+        const int item = int(blockIdx.x) + pit * int(gridDim.x);
+        const int64_t row0 = int64_t(item) * a.R;
+        const int rows_here = a.M - row0 < a.R ? static_cast<int>(a.M - row0) : a.R;
+        const unsigned long long* rmax = rowmax + (pit & 3) * kRqtMaxRows;
+        mbar_wait_bounded_lazy(&rowbar[pit & 3], static_cast<uint32_t>((pit >> 2) & 1), a.wait_limit_ns,
+                               abort_flag);
+        if (c < rows_here)  // one thread per row stores its scale s = s16 / 16
+          a.s_out[row0 + c] = __fmul_rn(div127(__uint_as_float(static_cast<uint32_t>(rmax[c]))), 0.0625f);
+        tmem_st_wait();
+#pragma unroll
+        for (int t = 0; t < GPS; ++t) {
+          uint32_t v[32];
+          tmem_ld32(tm + static_cast<uint32_t>(((pit & 1) * GPS + t) * 32), v);
+          tmem_ld_wait();
+          float2 u[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) u[i] = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          const float s16 = div127(__uint_as_float(static_cast<uint32_t>(rmax[rr[t]])));
+          if (act[t] && rr[t] < rows_here) {
+            const RowQuot rq = row_quotient(s16);
+            int8_t* out = a.q + (row0 + rr[t]) * a.K + 256 * gg[t] + 4 * l;
+            if (rq.f == 1.0f)
+              quantize_store<false>(u, rq, sel, out);
+            else
+              quantize_store<true>(u, rq, sel, out);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, a.tmem_cols);
+  }
+}
+
+// ----------------------------------------------------------------------------
 // Host side: shape choice and launch. The per-device host caches below (kernel
 // attributes set, chosen shape and occupancy per row length, SM count) are
 // read and written only under this mutex, which rotquant_plan holds.
@@ -603,6 +860,7 @@ RqArgs rotquant_args(const RqShape& sh, int64_t rows, int64_t K, int8_t* q, floa
   a.q = q;
   a.s_out = s;
   a.wait_limit_ns = wait_limit_ns;
+  a.tmem_cols = rotquant_tm_cols(sh.warps, sh.gps);
   return a;
 }
 
@@ -618,6 +876,167 @@ cudaError_t launch_rotquant(const CUtensorMap& tmap, const RqShape& sh, int occ,
     rotquant_kernel<T, 1><<<grid, threads, smem, stream>>>(tmap, a);
   else
     rotquant_kernel<T, 2><<<grid, threads, smem, stream>>>(tmap, a);
+  return cudaGetLastError();
+}
+
+// ---- host side of the tensor-memory variant
+template <typename T, int GPS>
+cudaError_t rotquant_tm_prepare_attr(int dev) {
+  static bool done[16] = {};
+  if (dev < 0 || dev >= 16) return cudaErrorInvalidDevice;
+  if (done[dev]) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(rotquant_tm_kernel<T, GPS>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
+
+// Blocks per SM of a kernel by registers, shared memory, threads and the block
+// limit, from its attributes and the device's. The runtime's occupancy query
+// reports one block per SM for these kernels, which allocate tensor memory, where
+// two fit and run (measured: both resident, x 80 -> 76 us at 16384 rows), so the
+// count is made here; the tensor-memory limit is applied by the caller.
+inline int blocks_per_sm_by_resources(const void* kernel, int threads, size_t dyn_smem, int dev) {
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return 0;
+  int regs_sm = 0, smem_sm = 0, reserved = 0, threads_sm = 0, blocks_sm = 0;
+  if (cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&threads_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&blocks_sm, cudaDevAttrMaxBlocksPerMultiprocessor, dev) != cudaSuccess)
+    return 0;
+  const int warps = (threads + 31) / 32;
+  const int regs_warp = ((fa.numRegs * 32 + 255) / 256) * 256;  // allocated per warp in units of 256
+  int n = blocks_sm;
+  if (regs_warp > 0) n = std::min(n, regs_sm / (regs_warp * warps));
+  n = std::min(n, threads_sm / (warps * 32));
+  const size_t smem_block = dyn_smem + fa.sharedSizeBytes + size_t(reserved);
+  n = std::min(n, int(size_t(smem_sm) / smem_block));
+  return n;
+}
+
+template <typename T>
+int rotquant_tm_occupancy(int gps, int threads, size_t smem, int dev) {
+  if (gps == 1) {
+    if (rotquant_tm_prepare_attr<T, 1>(dev) != cudaSuccess) return 0;
+    return blocks_per_sm_by_resources(reinterpret_cast<const void*>(rotquant_tm_kernel<T, 1>), threads, smem, dev);
+  }
+  if (rotquant_tm_prepare_attr<T, 2>(dev) != cudaSuccess) return 0;
+  return blocks_per_sm_by_resources(reinterpret_cast<const void*>(rotquant_tm_kernel<T, 2>), threads, smem, dev);
+}
+
+// Shape of the tensor-memory variant for rows of G = K / 256 groups: 1 or 2
+// groups per quarter-warp, up to 16 consumer warps, as many rows per item as the
+// quarters hold, 2 to 4 stages; blocks per SM limited by registers, shared memory
+// and the 512 tensor-memory columns of an SM. Kept: the most consumer warps doing
+// useful work per SM (two groups per quarter preferred: half the per-item work
+// per element), then the most bytes in flight. bf16 rows of K = 5376 use the shape
+// measured fastest (two groups per quarter, 8 consumer warps, 3 rows per item, 2
+// stages, two blocks per SM: 75.8 us at 16384 rows).
+// *smem_bytes: the dynamic shared memory to launch with. Where registers and
+// shared memory would let more blocks share an SM than its tensor memory holds,
+// the request is raised until they do not, so no block waits in tcgen05.alloc for
+// another block on its SM to finish.
+template <typename T>
+RqShape rotquant_tm_plan(int K, int dev, int* blocks_per_sm, int* sms, size_t* smem_bytes) {
+  std::lock_guard<std::mutex> lock(rotquant_host_mutex());
+  static RqShape cache[16][65] = {};
+  static int cache_occ[16][65] = {};
+  static size_t cache_smem[16][65] = {};
+  static int sm_count[16] = {};
+  *blocks_per_sm = 0;
+  *sms = 0;
+  *smem_bytes = 0;
+  if (dev < 0 || dev >= 16) return RqShape{0, 0, 0, 0};
+  if (sm_count[dev] == 0 &&
+      cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return RqShape{0, 0, 0, 0};
+  *sms = sm_count[dev];
+  const int G = K / 256;
+  if (G <= 64 && cache[dev][G].gps != 0) {
+    *blocks_per_sm = cache_occ[dev][G];
+    *smem_bytes = cache_smem[dev][G];
+    return cache[dev][G];
+  }
+  int n = 0, u = 0;
+  rotquant_copies<T>(K, &n, &u);
+  // blocks per SM (0 if the shape does not fit) and the shared memory to request
+  auto evaluate = [&](const RqShape& sh, size_t* launch_smem) -> int {
+    const uint32_t stage_bytes = uint32_t(n) * rotquant_copy_bytes<T>(K, sh.rows);
+    size_t smem = rotquant_tm_smem_bytes(sh.stages, stage_bytes, sh.warps);
+    if (smem > 227 * 1024) return 0;
+    const int threads = 32 * (sh.warps + 1);
+    const int by_tmem = int(512u / rotquant_tm_cols(sh.warps, sh.gps));
+    int occ = rotquant_tm_occupancy<T>(sh.gps, threads, smem, dev);
+    while (occ > by_tmem && smem + 1024 <= 227 * 1024) {
+      smem += 1024;
+      occ = rotquant_tm_occupancy<T>(sh.gps, threads, smem, dev);
+    }
+    if (occ > by_tmem) return 0;
+    *launch_smem = smem;
+    return occ;
+  };
+  RqShape best{0, 0, 0, 0};
+  int best_occ = 0;
+  size_t best_smem = 0;
+  if (sizeof(T) == 2 && G == 21) {
+    const RqShape pick{2, 8, 3, 2};
+    size_t sm = 0;
+    const int occ = evaluate(pick, &sm);
+    if (occ >= 1) {
+      best = pick;
+      best_occ = occ;
+      best_smem = sm;
+    }
+  }
+  double best_score = best.gps != 0 ? 1e30 : -1.0;
+  for (int gps = 2; gps >= 1 && best_score < 1e29; --gps)
+    for (int W = 1; W <= kRqtMaxWarps; ++W) {
+      const int slots = 4 * W * gps;
+      int R = slots / G;
+      if (R < 1) continue;
+      if (R > kRqtMaxRows) R = kRqtMaxRows;
+      if (rotquant_tm_cols(W, gps) > 512) continue;
+      const uint32_t stage_bytes = uint32_t(n) * rotquant_copy_bytes<T>(K, R);
+      for (int stages = 2; stages <= 4; ++stages) {
+        const RqShape sh{gps, W, R, stages};
+        size_t sm = 0;
+        const int occ = evaluate(sh, &sm);
+        if (occ < 1) break;
+        const double busy = double(R * G) / double(slots);
+        const double inflight = double(occ) * stages * stage_bytes;
+        const double score = occ * W * busy * (gps == 2 ? 1.1 : 1.0) +
+                             4.0 * (inflight < 131072.0 ? inflight : 131072.0) / 131072.0 - 0.001 * R;
+        if (score > best_score) {
+          best_score = score;
+          best = sh;
+          best_occ = occ;
+          best_smem = sm;
+        }
+      }
+    }
+  if (G <= 64 && best.gps != 0) {
+    cache[dev][G] = best;
+    cache_occ[dev][G] = best_occ;
+    cache_smem[dev][G] = best_smem;
+  }
+  *blocks_per_sm = best_occ;
+  *smem_bytes = best_smem;
+  return best;
+}
+
+// Launches a tensor-memory plan: a persistent grid of min(items, SMs x blocks per SM) blocks.
+template <typename T>
+cudaError_t launch_rotquant_tm(const CUtensorMap& tmap, const RqShape& sh, int occ, int sms, size_t smem,
+                               const RqArgs& a, cudaStream_t stream) {
+  const int threads = 32 * (sh.warps + 1);
+  const int64_t cap = int64_t(sms) * occ;
+  const unsigned grid = static_cast<unsigned>(a.items < cap ? a.items : cap);
+  if (sh.gps == 1)
+    rotquant_tm_kernel<T, 1><<<grid, threads, smem, stream>>>(tmap, a);
+  else
+    rotquant_tm_kernel<T, 2><<<grid, threads, smem, stream>>>(tmap, a);
   return cudaGetLastError();
 }
 
