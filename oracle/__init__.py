@@ -356,15 +356,16 @@ def nvfp4_epilogue(acc32, s_enc_a, s_enc_w, bias_bits=None, swiglu_epilogue=Fals
 # ------------------------------------------------------------ int8 attention
 def attention_int8(q_bits, k_bits, v_bits, H, D=128, rows=None):
     """int8 Q.K^T / softmax / P.V per head. q, k, v: bf16 bits [S, ld], head h at
-    columns h*D .. h*D+D-1. Returns (o float64 [n, H*D] for the query rows
-    `rows` (all rows if None), qq int8 [H, S, D], qs fp32 [H, S], kq, ks)."""
+    columns h*D .. h*D+D-1. Q is quantized per token, K per block of 128 keys.
+    Returns (o float64 [n, H*D] for the query rows `rows` (all rows if None),
+    qq int8 [H, S, D], qs fp32 [H, S], kq int8 [H, S, D], ks fp32 [H, ceil(S/128)])."""
     q, k, v = (_c(a, np.uint16) for a in (q_bits, k_bits, v_bits))
     assert q.shape == k.shape == v.shape and q.shape[1] >= H * D
     S, ld = q.shape
     qq = np.empty((H, S, D), dtype=np.int8)
     kq = np.empty((H, S, D), dtype=np.int8)
     qs = np.empty((H, S), dtype=np.float32)
-    ks = np.empty((H, S), dtype=np.float32)
+    ks = np.empty((H, (S + 127) // 128), dtype=np.float32)
     r = None if rows is None else _c(rows, np.int64)
     n = S if r is None else r.size
     o = np.empty((n, H * D), dtype=np.float64)

@@ -38,6 +38,7 @@
 // Plain loops, no blocking or fusion beyond what the definition states.
 // Build: g++ -O2 -std=c++17 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -534,12 +535,16 @@ void orc_nvfp4_linear(const uint8_t* ca, const uint8_t* sfa, float s_enc_a, int6
 // int8 attention (h3-rs README, "What makes it fast": the DiT attention runs an
 // int8 Q.K^T / 16-bit P.V flash kernel). Per head h (columns h*D .. h*D+D-1 of
 // the [S, ld] q, k, v matrices, bf16 bit patterns):
-//   Q and K rows (one token of one head) are quantized like weight rows
-//   (steps 3-4: s = max|x| / 127 in fp32, codes clamp(rne(x / s)));
-//   s_ij = (sum_d Qq_id Kq_jd) * qs_i * ks_j / sqrt(D)   (exact integer dot product)
-//   O_i  = sum_j softmax_j(s_i)_j V_j                      (float64)
-// qq, kq [H, S, D] int8 and qs, ks [H, S]; o [n, H*D] float64 for the query
-// rows rows[0..n) (all S rows in order when rows is null).
+//   Q rows (one token of one head) are quantized like weight rows (steps 3-4:
+//   s = max|x| / 127 in fp32, codes clamp(rne(x / s)));
+//   K is quantized in blocks of 128 consecutive keys of a head: one scale per
+//   block, s = max|x| / 127 over the block's keys and dimensions, codes
+//   clamp(rne(x / s)) (steps 3-4 on the block read as one vector; the last
+//   block of a sequence takes the keys that remain);
+//   s_ij = (sum_d Qq_id Kq_jd) * qs_i * ks_b(j) / sqrt(D)   (exact integer dot product)
+//   O_i  = sum_j softmax_j(s_i)_j V_j                        (float64)
+// qq, kq [H, S, D] int8, qs [H, S], ks [H, ceil(S / 128)]; o [n, H*D] float64 for
+// the query rows rows[0..n) (all S rows in order when rows is null).
 // ---------------------------------------------------------------------------
 void orc_attention_int8(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S, int64_t D, int64_t H,
                         int64_t ld, int8_t* qq, float* qs, int8_t* kq, float* ks, const int64_t* rows, int64_t n,
@@ -551,8 +556,15 @@ void orc_attention_int8(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     std::vector<float> row(D);
     for (int64_t d = 0; d < D; ++d) row[d] = bf16_to_f32(q[i * ld + h * D + d]);
     quantize_row(row.data(), D, qq + t * D, qs + t);
-    for (int64_t d = 0; d < D; ++d) row[d] = bf16_to_f32(k[i * ld + h * D + d]);
-    quantize_row(row.data(), D, kq + t * D, ks + t);
+  }
+  const int64_t kb = 128, nblk = (S + kb - 1) / kb;
+#pragma omp parallel for schedule(static)
+  for (int64_t u = 0; u < H * nblk; ++u) {
+    const int64_t h = u / nblk, b = u % nblk, j0 = b * kb, nk = std::min(kb, S - j0);
+    std::vector<float> blk(nk * D);
+    for (int64_t j = 0; j < nk; ++j)
+      for (int64_t d = 0; d < D; ++d) blk[j * D + d] = bf16_to_f32(k[(j0 + j) * ld + h * D + d]);
+    quantize_row(blk.data(), nk * D, kq + (h * S + j0) * D, ks + u);
   }
   const double inv_sqrt_d = 1.0 / std::sqrt(double(D));
 #pragma omp parallel for schedule(dynamic, 1)
@@ -565,7 +577,7 @@ void orc_attention_int8(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     for (int64_t j = 0; j < S; ++j) {
       int64_t dot = 0;
       for (int64_t d = 0; d < D; ++d) dot += int64_t(qq[t * D + d]) * int64_t(kq[(h * S + j) * D + d]);
-      sc[j] = double(dot) * double(qs[t]) * double(ks[h * S + j]) * inv_sqrt_d;
+      sc[j] = double(dot) * double(qs[t]) * double(ks[h * nblk + j / kb]) * inv_sqrt_d;
       mx = std::fmax(mx, sc[j]);
     }
     double l = 0.0;

@@ -29,14 +29,38 @@ def _inputs(S, H, seed, outlier=True):
     return _bits(q), _bits(k), _bits(v)
 
 
-def test_codes_are_the_row_quantizer_per_head():
-    q, k, v = _inputs(40, 2, 0)
-    _, qq, qs, kq, ks = oracle.attention_int8(q, k, v, 2)
-    for h in range(2):
+def test_codes_q_per_token_k_per_block_of_128_keys():
+    """Q rows use the weight-row quantizer per token; K uses it per block of 128 keys
+    of a head (the block read as one vector), the last block taking the keys left."""
+    S, H = 300, 2  # key blocks of 128, 128 and 44
+    q, k, v = _inputs(S, H, 0)
+    _, qq, qs, kq, ks = oracle.attention_int8(q, k, v, H)
+    assert ks.shape == (H, 3)
+    for h in range(H):
         cq, sq = oracle.quantize_rows(_vals(q[:, h * D:(h + 1) * D]).astype(np.float32))
         assert np.array_equal(qq[h], cq) and np.array_equal(qs[h], sq)
-        ck, sk = oracle.quantize_rows(_vals(k[:, h * D:(h + 1) * D]).astype(np.float32))
-        assert np.array_equal(kq[h], ck) and np.array_equal(ks[h], sk)
+        kh = _vals(k[:, h * D:(h + 1) * D]).astype(np.float32)
+        for b, (j0, j1) in enumerate(((0, 128), (128, 256), (256, 300))):
+            ck, sk = oracle.quantize_rows(kh[j0:j1].reshape(1, -1))
+            assert np.array_equal(kq[h, j0:j1], ck.reshape(j1 - j0, D)) and ks[h, b] == sk[0]
+
+
+def test_key_block_scale_covers_its_own_block_only():
+    """Doubling the keys of block 1 (exact in bf16) doubles its scale and keeps its
+    codes; block 0 is untouched; one large key coarsens only its own block."""
+    S = 256
+    q, k, v = _inputs(S, 1, 5, outlier=False)
+    _, _, _, kq, ks = oracle.attention_int8(q, k, v, 1)
+    k2 = k.copy()
+    k2[128:] = _bits(_vals(k[128:]) * 2.0)
+    _, _, _, kq2, ks2 = oracle.attention_int8(q, k2, v, 1)
+    assert ks2[0, 0] == ks[0, 0] and ks2[0, 1] == 2 * ks[0, 1]
+    assert np.array_equal(kq2, kq)
+    k3 = k.copy()
+    k3[200, 3] = _bits(np.array([[1000.0]]))[0, 0]
+    _, _, _, kq3, ks3 = oracle.attention_int8(q, k3, v, 1)
+    assert ks3[0, 0] == ks[0, 0] and np.array_equal(kq3[0, :128], kq[0, :128])
+    assert ks3[0, 1] > 100 * ks[0, 1] and kq3[0, 200, 3] == 127
 
 
 def test_identical_keys_give_the_mean_of_v():
@@ -47,11 +71,12 @@ def test_identical_keys_give_the_mean_of_v():
 
 
 def test_matches_torch_sdpa_on_dequantized_inputs():
-    S, H = 70, 3
+    S, H = 200, 3
     q, k, v = _inputs(S, H, 2)
     o, qq, qs, kq, ks = oracle.attention_int8(q, k, v, H)
     qd = torch.from_numpy(qq.astype(np.float64) * qs[:, :, None].astype(np.float64))
-    kd = torch.from_numpy(kq.astype(np.float64) * ks[:, :, None].astype(np.float64))
+    ks_key = np.repeat(ks.astype(np.float64), 128, axis=1)[:, :S]  # each key's block scale
+    kd = torch.from_numpy(kq.astype(np.float64) * ks_key[:, :, None])
     vd = torch.from_numpy(_vals(v).reshape(S, H, D).transpose(1, 0, 2).copy())
     ref = torch.nn.functional.scaled_dot_product_attention(qd[None], kd[None], vd[None])[0]
     ref = ref.numpy().transpose(1, 0, 2).reshape(S, H * D)
