@@ -223,9 +223,11 @@ h3q_status h3q_gemm_nvfp4_f32(const uint8_t* xc, const uint8_t* xsf, int64_t M, 
  * int8 Q.K^T / 16-bit P.V flash kernel). Head dim 128; head h of q, k, v and out
  * is columns h*128 .. h*128+127 of a row-major [S, ld] bf16 matrix (q, k and v
  * may be column slices of one QKV projection output).
- *   Q and K rows (one token of one head) are quantized like weight rows:
- *   s = max|x| / 127 (fp32), codes clamp(rne(x / s));
- *   s_ij = (sum_d Qq_id Kq_jd) qs_i ks_j / sqrt(128); O_i = softmax_j(s_i) V;
+ *   Q rows (one token of one head) are quantized like weight rows: s = max|x| /
+ *   127 (fp32), codes clamp(rne(x / s)); K is quantized the same way per block
+ *   of 128 consecutive keys of a head (one scale over the block's keys and
+ *   dimensions; the last block takes the keys that remain);
+ *   s_ij = (sum_d Qq_id Kq_jd) qs_i ks_b(j) / sqrt(128); O_i = softmax_j(s_i) V;
  *   P is rounded to bf16 and P.V accumulated in fp32 (the hardware's order);
  *   out = bf16(O).
  * workspace: h3q_attention_workspace_size(S, H) bytes, 256-byte aligned (codes,
@@ -239,7 +241,8 @@ h3q_status h3q_attention_int8(const void* q, const void* k, const void* v, int64
 
 /*
  * The attention's input pass on its own (test hook and building block): qq, kq
- * int8 [H, S, 128], qs, ks fp32 [H, S], vt bf16 [H*128, S] (V^T per head).
+ * int8 [H, S, 128], qs fp32 [H, S], ks fp32 [H, ceil(S / 128)] (one per block of
+ * 128 keys), vt bf16 [H*128, S] (V^T per head).
  */
 h3q_status h3q_attention_prep(const void* q, const void* k, const void* v, int64_t S, int64_t H, int64_t ld,
                               int8_t* qq, float* qs, int8_t* kq, float* ks, void* vt, cudaStream_t stream);

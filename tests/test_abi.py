@@ -143,7 +143,7 @@ def test_nvfp4_sizes_and_rejects():
 def test_attention_rejects():
     f = h3q.lib.h3q_attention_int8
     ws = h3q.h3q_attention_workspace_size(64, 2)
-    assert ws >= 2 * 64 * 128 * 4 + 2 * 2 * 64 * 4
+    assert ws >= 2 * 64 * 128 * 4 + 2 * 64 * 4 + 2 * 4  # codes, V^T, qs [H, S], ks [H, S / 128]
     ok = [FAKE, FAKE, FAKE, 64, 2, 256, FAKE, 256, FAKE, ws, None]
     for i, bad in [(3, 60), (4, 0), (5, 200), (5, 260), (7, 100), (9, ws - 1), (8, FAKE + 16), (0, None),
                    (6, FAKE + 8)]:

@@ -1,7 +1,7 @@
 """int8 attention on the GPU against the oracle.
 
-* The input pass (per-token int8 codes and scales of Q and K per head, V^T) is
-  bit-exact.
+* The input pass (int8 codes of Q per token and of K per block of 128 keys, their
+  scales, V^T per head) is bit-exact.
 * The attention output is compared with the oracle's float64 attention of the
   same int8 codes within a bound from the arithmetic: P is rounded to bf16
   (relative 2^-9 per weight, the row sum uses the same rounded weights, so the
@@ -68,7 +68,7 @@ def test_prep_is_bit_exact(cuda_device):
     qq = torch.empty((H, S, D), dtype=torch.int8, device=cuda_device)
     kq = torch.empty_like(qq)
     qs = torch.empty((H, S), dtype=torch.float32, device=cuda_device)
-    ks = torch.empty_like(qs)
+    ks = torch.empty((H, (S + 127) // 128), dtype=torch.float32, device=cuda_device)
     vt = torch.empty((H * D, S), dtype=torch.bfloat16, device=cuda_device)
     h3q.h3q_attention_prep(q, k, v, H, qq, qs, kq, ks, vt)
     torch.cuda.synchronize()

@@ -302,14 +302,15 @@ def h3q_attention_int8(q, k, v, H, out, workspace, stream=None) -> None:
 
 
 def h3q_attention_prep(q, k, v, H, qq, qs, kq, ks, vt, stream=None) -> None:
-    """The attention's input pass: int8 Q/K codes and scales per head, V^T per head."""
+    """The attention's input pass: int8 Q codes and scales per token and head, K codes per
+    head with one scale per block of 128 keys (ks [H, ceil(S/128)]), V^T per head."""
     w = "h3q_attention_prep"
     S = _attention_inputs(w, q, k, v, H)
     dev = q.device
     _need(w, "qq", qq, "i8", (H, S, 128), dev)
     _need(w, "kq", kq, "i8", (H, S, 128), dev)
     _need(w, "qs", qs, "f32", (H, S), dev)
-    _need(w, "ks", ks, "f32", (H, S), dev)
+    _need(w, "ks", ks, "f32", (H, (S + 127) // 128), dev)
     _need(w, "vt", vt, "bf16", (H * 128, S), dev)
     _check(lib.h3q_attention_prep(_ptr(q), _ptr(k), _ptr(v), S, H, _ld(q), _ptr(qq), _ptr(qs), _ptr(kq), _ptr(ks),
                                   _ptr(vt), _stream(stream)), "h3q_attention_prep")

@@ -1,20 +1,21 @@
 // int8 attention for the DiT blocks (h3-rs README, "What makes it fast": an
 // int8 Q.K^T / 16-bit P.V flash kernel). Per head (head dim 128, columns
 // h*128 .. h*128+127 of the [S, ld] q, k, v and out matrices):
-//   Q and K rows are quantized per token (s = max|x| / 127 in fp32, codes
-//   clamp(rne(x / s)), as the weight rows of the linear layers);
-//   s_ij = acc_ij * qs_i * ks_j / sqrt(128) with acc the exact int32 dot product;
+//   Q rows are quantized per token (s = max|x| / 127 in fp32, codes
+//   clamp(rne(x / s)), as the weight rows of the linear layers), K per block of
+//   128 consecutive keys (one scale over the block's keys and dimensions), so the
+//   key scale is one constant per key tile;
+//   s_ij = acc_ij * qs_i * ks_b(j) / sqrt(128) with acc the exact int32 dot product;
 //   O_i = softmax_j(s_i) V, with P in bf16 and fp32 accumulation.
 //
-// attn_prep_kernel: one block per (64-token tile, head): Q and K codes and
-// scales, and V transposed per head (V^T [H*128, S]) so both products read
-// K-major operands.
+// attn_prep_kernel: one block per (128-token tile, head): Q codes and scales per
+// token, the tile's K codes with its one scale, and V transposed per head (V^T
+// [H*128, S]) so both products read K-major operands.
 //
 // attn_kernel: one CTA per (head, 128-query block); warp roles:
 //   warp 0   TMA: the Q tile once, then per block of 128 keys the K tile (a
 //            three-stage ring, released once S_j = Q K_j^T is done) and the
-//            V^T tile with the key scales (a three-stage ring, released once
-//            P_j V_j is done);
+//            V^T tile (a three-stage ring, released once P_j V_j is done);
 //   warp 1   tensor memory (512 columns: two 128-column score buffers, the
 //            128-column output accumulator O and two 64-column P buffers);
 //            one lane issues O += P_j V_j (kind::f16, A = P_j from tensor
@@ -26,9 +27,10 @@
 //   warps 4-11 softmax, two sets of four warps, one thread per query row
 //            (tensor-memory lane): set 0 takes the even key blocks, set 1 the
 //            odd ones, so one set's exponentials overlap the other's score
-//            loads. For its block a thread reads the whole score row, scales
-//            it with the key scales, takes the row maximum, and writes
-//            P = 2^(s - m) as bf16 into P buffer j % 2. The maximum m used in
+//            loads. For its block a thread reads the whole score row, takes
+//            its maximum, and writes P = 2^(s - m) as bf16 into P buffer j % 2,
+//            the block's key scale folded into one multiply-add per key. The
+//            maximum m used in
 //            the exponent is handed from block to block through shared memory
 //            (the set of block j publishes it, the set of block j+1 waits for
 //            it); it is raised only when a row's maximum grows by more than
@@ -54,7 +56,7 @@ constexpr int kAttQBytes = 128 * 128;      // int8 Q tile
 constexpr int kAttKBytes = 128 * 128;      // int8 K tile
 constexpr int kAttVBytes = 2 * 128 * 128;  // bf16 V^T tile (128 d rows x 128 keys), two 64-key boxes
 constexpr int kAttKStages = 3;  // K ring: K_{j+3} loads once S_j = Q K_j^T is done
-constexpr int kAttVStages = 3;  // V^T ring (with the key scales): V_{j+3} loads once P_j V_j is done
+constexpr int kAttVStages = 3;  // V^T ring: V_{j+3} loads once P_j V_j is done
 constexpr int kAttThreads = 128 + 2 * 128;  // producer, MMA (and two idle warps), two softmax sets
 // Register split (setmaxnreg): the first warpgroup gives registers back, the two
 // softmax warpgroups take them. The kernel is launched with at least
@@ -62,20 +64,19 @@ constexpr int kAttThreads = 128 + 2 * 128;  // producer, MMA (and two idle warps
 // the split never asks for more than the block holds.
 constexpr uint32_t kAttRegsCtl = 40, kAttRegsSoftmax = 232, kAttRegsLaunch = 168;
 static_assert(128 * kAttRegsCtl + 256 * kAttRegsSoftmax <= kAttThreads * kAttRegsLaunch, "register split");
-constexpr int kAttKsBytes = 128 * 4;       // the key block's scales
 // tensor-memory columns
 constexpr uint32_t kAttColS = 0;    // score buffers b at b * 128 (int32)
 constexpr uint32_t kAttColO = 256;  // output accumulator (fp32)
 constexpr uint32_t kAttColP = 384;  // P buffers b at 384 + b * 64 (bf16 pairs)
 constexpr int kAttBiasBytes = 2 * 128 * 128;  // the bias product's two bf16 operands (128 x 64, swizzled)
 constexpr size_t kAttSmem = size_t(kAttBiasBytes) + kAttQBytes + kAttKStages * kAttKBytes +
-                            kAttVStages * (size_t(kAttVBytes) + kAttKsBytes) + 2 * 128 * 4 /*maxima*/ +
+                            kAttVStages * size_t(kAttVBytes) + 2 * 128 * 4 /*maxima*/ +
                             2 * 128 * 4 /*row sums*/ + 1024 + 256;
 
 struct AttParams {
   int S, H;
   const float* qs;       // [H, S]
-  const float* ks;       // [H, S]
+  const float* ks;       // [H, ceil(S / 128)]: one scale per block of 128 keys
   __nv_bfloat16* out;    // [S, ld_out], head h at columns h*128
   int64_t ld_out;
   float c;               // log2(e) / sqrt(128)
@@ -137,47 +138,43 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Scales a block's raw scores in place, s'_k = (float)acc_k * ks_k, and returns
-// their maximum. The accumulators start from the fp32 bits of 1.5 * 2^23 (written
-// by a bf16 product before the int8 ones), so they hold 0x4B400000 + acc; with
-// |acc| <= 127^2 * 128 < 2^22 those bits read as a float are 1.5 * 2^23 + acc
-// exactly, and one subtraction gives (float)acc, without the conversion unit. With kMasked, keys k >= nvalid (past the end of the
-// sequence) get s' = -inf; the two forms are separate so the unmasked one,
-// used for every block but the last, carries no per-key predicates.
+// The block's raw scores: the score products accumulate onto the bits of the fp32
+// value 1.5 * 2^23 (written first by one bf16 product), and |acc| <= 127^2 * 128 <
+// 2^22, so each column read as a float is F = 1.5 * 2^23 + acc exactly. Keys past
+// the end (last block only) are set to -inf. Returns the largest F of the row.
 template <bool kMasked>
-__device__ __forceinline__ float att_scores(uint32_t (&sr)[4][32], const float* ksb, int nvalid) {
-  const float2 magic2 = make_float2(-12582912.0f, -12582912.0f);
+__device__ __forceinline__ float att_raw_max(uint32_t (&sr)[4][32], int nvalid) {
   float mx = -INFINITY;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
 #pragma unroll
     for (int e4 = 0; e4 < 8; ++e4) {
       const int k0 = 4 * e4;
-      const float4 kv = *reinterpret_cast<const float4*>(ksb + 32 * c + k0);
-      float2 x01 = make_float2(__uint_as_float(sr[c][k0]), __uint_as_float(sr[c][k0 + 1]));
-      float2 x23 = make_float2(__uint_as_float(sr[c][k0 + 2]), __uint_as_float(sr[c][k0 + 3]));
-      x01 = __fmul2_rn(__fadd2_rn(x01, magic2), make_float2(kv.x, kv.y));
-      x23 = __fmul2_rn(__fadd2_rn(x23, magic2), make_float2(kv.z, kv.w));
-      float sc[4] = {x01.x, x01.y, x23.x, x23.y};
+      float sc[4] = {__uint_as_float(sr[c][k0]), __uint_as_float(sr[c][k0 + 1]), __uint_as_float(sr[c][k0 + 2]),
+                     __uint_as_float(sr[c][k0 + 3])};
       if (kMasked) {
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (32 * c + k0 + e >= nvalid) sc[e] = -INFINITY;
+          if (32 * c + k0 + e >= nvalid) {
+            sc[e] = -INFINITY;
+            sr[c][k0 + e] = __float_as_uint(-INFINITY);
+          }
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sr[c][k0 + e] = __float_as_uint(sc[e]);
       mx = att_max3(mx, att_max3(sc[0], sc[1], sc[2]), sc[3]);
     }
   }
   return mx;
 }
 
-// P_k = 2^(s'_k cq - m cq) as bf16 pairs (lower key in the low half) into the
-// 64 P columns at p_cols; returns the sum of the (unrounded) weights. With
-// kMasked, keys k >= nvalid weigh 0 (also when cq = 0, where -inf * cq is not a
-// number).
+// P_k = 2^(F_k c - b) as bf16 pairs (lower key in the low half) into the 64 P
+// columns at p_cols, F_k the raw scores of att_raw_max, c = RN(ks cq) and b =
+// RN(RN(1.5 * 2^23 c) + RN(m cq)): the exponent (acc_k ks - m) cq in one fused
+// multiply-add per key (F_k c is exact inside it; b differs from the exact bias by
+// about one unit of acc_k c, well below the bf16 rounding of P). Returns the sum
+// of the (unrounded) weights. With kMasked, keys k >= nvalid weigh 0 (also when
+// c = 0, where -inf * c is not a number).
 template <bool kMasked>
-__device__ __forceinline__ float2 att_weights(const uint32_t (&sr)[4][32], float2 cq2, float2 nm2, int nvalid,
+__device__ __forceinline__ float2 att_weights(const uint32_t (&sr)[4][32], float2 c2, float2 nb2, int nvalid,
                                               uint32_t p_cols) {
   float2 bs2 = make_float2(0.0f, 0.0f);
 #pragma unroll
@@ -187,7 +184,7 @@ __device__ __forceinline__ float2 att_weights(const uint32_t (&sr)[4][32], float
     for (int e = 0; e < 32; ++e) {
       const int k0 = 64 * hh + 2 * e;
       const float2 t = __ffma2_rn(
-          make_float2(__uint_as_float(sr[k0 >> 5][k0 & 31]), __uint_as_float(sr[k0 >> 5][(k0 & 31) + 1])), cq2, nm2);
+          make_float2(__uint_as_float(sr[k0 >> 5][k0 & 31]), __uint_as_float(sr[k0 >> 5][(k0 & 31) + 1])), c2, nb2);
       float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
       if (kMasked) {
         if (k0 >= nvalid) p0 = 0.0f;
@@ -202,45 +199,82 @@ __device__ __forceinline__ float2 att_weights(const uint32_t (&sr)[4][32], float
 }
 
 // ---------------------------------------------------------------- prep
-// Block (tile of 64 tokens, head h), 256 threads. Q/K rows: one warp per token
-// (4 elements per lane); V: staged in shared memory and written transposed.
+// Block (tile of 128 tokens = one key block, head h), 256 threads. Q rows: one
+// warp per token (4 elements per lane), a scale per token. K: the tile's max|x|
+// over its keys and dimensions gives the block's one scale, then each key row is
+// quantized with it (read again, from L1/L2). V: staged in shared memory and
+// written transposed.
+__device__ __forceinline__ void att_load4(const __nv_bfloat16* src, float (&x)[4]) {
+  const uint2 w = *reinterpret_cast<const uint2*>(src);
+  x[0] = __uint_as_float(w.x << 16);
+  x[1] = __uint_as_float(w.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(w.y << 16);
+  x[3] = __uint_as_float(w.y & 0xFFFF0000u);
+}
+
+// Four int8 codes clamp(rne(x / s)) packed in a word (0 where s = 0).
+__device__ __forceinline__ uint32_t att_codes4(const float (&x)[4], float s) {
+  uint32_t packed = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float r = 0.0f;
+    if (s != 0.0f) r = fminf(fmaxf(rintf(__fdiv_rn(x[e], s)), -127.0f), 127.0f);
+    packed |= (static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu) << (8 * e);
+  }
+  return packed;
+}
+
 __global__ void __launch_bounds__(256) attn_prep_kernel(const __nv_bfloat16* __restrict__ q,
                                                         const __nv_bfloat16* __restrict__ k,
                                                         const __nv_bfloat16* __restrict__ v, int S, int64_t ld,
                                                         int8_t* __restrict__ qq, float* __restrict__ qs,
                                                         int8_t* __restrict__ kq, float* __restrict__ ks,
                                                         __nv_bfloat16* __restrict__ vt) {
-  __shared__ uint16_t tile[64][kAttD + 2];  // +2 halves: column reads spread over banks
+  __shared__ uint16_t tile[kAttBlk][kAttD + 2];  // +2 halves: column reads spread over banks
+  __shared__ float warp_max[8];
   const int h = blockIdx.y;
-  const int t0 = blockIdx.x * 64;
+  const int t0 = blockIdx.x * kAttBlk;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int t = warp; t < 64; t += 8) {
+  // Q: a scale per token
+  for (int t = warp; t < kAttBlk; t += 8) {
     const int i = t0 + t;
     if (i >= S) break;
+    float x[4];
+    att_load4(q + int64_t(i) * ld + h * kAttD + 4 * lane, x);
+    float a = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const __nv_bfloat16* src = (which == 0 ? q : k) + int64_t(i) * ld + h * kAttD + 4 * lane;
-      const uint2 w = *reinterpret_cast<const uint2*>(src);
-      const float x[4] = {__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u),
-                          __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u)};
-      float a = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
-      const float s = __fdiv_rn(a, 127.0f);
-      uint32_t packed = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float r = 0.0f;
-        if (s != 0.0f) r = fminf(fmaxf(rintf(__fdiv_rn(x[e], s)), -127.0f), 127.0f);
-        packed |= (static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu) << (8 * e);
-      }
-      const int64_t row = int64_t(h) * S + i;
-      *reinterpret_cast<uint32_t*>((which == 0 ? qq : kq) + row * kAttD + 4 * lane) = packed;
-      if (lane == 0) (which == 0 ? qs : ks)[row] = s;
-    }
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+    const float sq = __fdiv_rn(a, 127.0f);
+    const int64_t row = int64_t(h) * S + i;
+    *reinterpret_cast<uint32_t*>(qq + row * kAttD + 4 * lane) = att_codes4(x, sq);
+    if (lane == 0) qs[row] = sq;
   }
-  // V tile [64 tokens][128 d] -> V^T rows h*128 + d, columns t0 .. t0+63
-  for (int e = threadIdx.x; e < 64 * (kAttD / 2); e += 256) {
+  // K: one scale for the tile's keys
+  float a = 0.0f;
+  for (int t = warp; t < kAttBlk; t += 8) {
+    const int i = t0 + t;
+    if (i >= S) break;
+    float x[4];
+    att_load4(k + int64_t(i) * ld + h * kAttD + 4 * lane, x);
+    a = fmaxf(a, fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  if (lane == 0) warp_max[warp] = a;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < 8; ++w) a = fmaxf(a, warp_max[w]);
+  const float sk = __fdiv_rn(a, 127.0f);
+  if (threadIdx.x == 0) ks[int64_t(h) * gridDim.x + blockIdx.x] = sk;
+  for (int t = warp; t < kAttBlk; t += 8) {
+    const int i = t0 + t;
+    if (i >= S) break;
+    float x[4];
+    att_load4(k + int64_t(i) * ld + h * kAttD + 4 * lane, x);
+    *reinterpret_cast<uint32_t*>(kq + (int64_t(h) * S + i) * kAttD + 4 * lane) = att_codes4(x, sk);
+  }
+  // V tile [128 tokens][128 d] -> V^T rows h*128 + d, columns t0 .. t0+127
+  for (int e = threadIdx.x; e < kAttBlk * (kAttD / 2); e += 256) {
     const int t = e / (kAttD / 2), d2 = e % (kAttD / 2);
     const int i = t0 + t;
     uint32_t w = 0;
@@ -249,8 +283,8 @@ __global__ void __launch_bounds__(256) attn_prep_kernel(const __nv_bfloat16* __r
     tile[t][2 * d2 + 1] = static_cast<uint16_t>(w >> 16);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kAttD * 32; e += 256) {
-    const int d = e / 32, t2 = e % 32;  // tokens 2 t2, 2 t2 + 1
+  for (int e = threadIdx.x; e < kAttD * (kAttBlk / 2); e += 256) {
+    const int d = e / (kAttBlk / 2), t2 = e % (kAttBlk / 2);  // tokens 2 t2, 2 t2 + 1
     const int i = t0 + 2 * t2;
     if (i >= S) continue;
     const uint32_t w = uint32_t(tile[2 * t2][d]) | (uint32_t(tile[2 * t2 + 1][d]) << 16);
@@ -268,14 +302,14 @@ __global__ void __launch_bounds__(kAttThreads, 1)
   uint8_t* sQ = sBias + kAttBiasBytes;
   uint8_t* sK = sQ + kAttQBytes;                   // [K stage][128 keys x 128 B]
   uint8_t* sV = sK + kAttKStages * kAttKBytes;     // [V stage][2 boxes: 128 d rows x 64 keys (128 B)]
-  float* sKs = reinterpret_cast<float*>(sV + kAttVStages * kAttVBytes);  // [V stage][128] key scales
-  float* sMx = sKs + kAttVStages * 128;            // [block parity][128 rows]: the maximum after a block
+  float* sMx = reinterpret_cast<float*>(sV + kAttVStages * kAttVBytes);  // [block parity][128 rows]:
+                                                                         // the maximum after a block
   float* sL = sMx + 2 * 128;                       // [set][128 rows]: the sets' row sums at the end
   uint64_t* bars = reinterpret_cast<uint64_t*>(sL + 2 * 128);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;    // [K stage]
   uint64_t* k_empty = bars + 4;   // [K stage]
-  uint64_t* v_full = bars + 7;    // [V stage]: V^T and the key scales
+  uint64_t* v_full = bars + 7;    // [V stage]: V^T
   uint64_t* v_empty = bars + 10;  // [V stage]
   uint64_t* s_full = bars + 13;   // [score buffer]
   uint64_t* s_empty = bars + 15;  // [score buffer]: its scores are in the softmax threads' registers
@@ -358,9 +392,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
           if (!mbar_wait_bounded(&v_empty[vst], static_cast<uint32_t>(((j / kAttVStages) & 1) ^ 1), limit,
                                  abort_flag))
             break;
-          const uint32_t ks_bytes = static_cast<uint32_t>(min(kAttBlk, S - j * kAttBlk) * 4);  // S % 8 == 0
-          mbar_arrive_expect_tx(&v_full[vst], kAttVBytes + ks_bytes);
-          bulk_load(sKs + vst * 128, p.ks + int64_t(h) * S + j * kAttBlk, ks_bytes, &v_full[vst], pol_kv);
+          mbar_arrive_expect_tx(&v_full[vst], kAttVBytes);
           tma_load_2d(sV + vst * kAttVBytes, &tmV, &v_full[vst], j * kAttBlk, h * kAttD, pol_kv);
           tma_load_2d(sV + vst * kAttVBytes + kAttVBytes / 2, &tmV, &v_full[vst], j * kAttBlk + 64, h * kAttD, pol_kv);
           ++nv;
@@ -463,16 +495,17 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[b]);  // S_{j+2} may now be written into buffer b
-      // Raw scores s' = (float)acc * ks_j (|acc| <= 127^2 * 128 < 2^22, so the bits of
-      // acc + 1.5 * 2^23 read as a float, minus 1.5 * 2^23, are (float)acc without the
-      // conversion unit); the log2-domain score is s' * cq, cq = qs_i log2(e) / sqrt(128) >= 0,
-      // so maxima can be taken on s'. Keys past the end (last block only) are masked.
+      // Scores s' = acc * ks_j (ks_j the key block's scale); the log2-domain score is
+      // s' * cq, cq = qs_i log2(e) / sqrt(128) >= 0, so maxima can be taken on s', and
+      // on the raw scores F = 1.5 * 2^23 + acc (ks_j >= 0). Keys past the end (last
+      // block only) are masked.
       if (!(ok = wait_all(&v_full[vst], static_cast<uint32_t>((j / kAttVStages) & 1)))) break;
-      const float* ksb = sKs + vst * 128;
+      const float ksj = __ldg(p.ks + int64_t(h) * nb + j);
       const int key0 = j * kAttBlk;
       const bool partial = key0 + kAttBlk > S;
       const int nvalid = S - key0;  // keys of the block inside the sequence (>= 8)
-      const float mx = partial ? att_scores<true>(sr, ksb, nvalid) : att_scores<false>(sr, ksb, nvalid);
+      const float f_max = partial ? att_raw_max<true>(sr, nvalid) : att_raw_max<false>(sr, nvalid);
+      const float mx = __fmul_rn(__fsub_rn(f_max, 12582912.0f), ksj);
       if (j > 0) {  // the maximum after block j-1, published by the other set
         if (!(ok = wait_all(&mx_full[(j - 1) & 1], static_cast<uint32_t>(((j - 1) >> 1) & 1)))) break;
         adopt(sMx[((j - 1) & 1) * 128 + r]);
@@ -488,11 +521,12 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       }
       tc_fence_after();
       // P = 2^(s' cq - m cq) as bf16 pairs (lower key in the low half), 64 keys per store
-      const float nm = -__fmul_rn(m_new, cq);
-      const float2 cq2 = make_float2(cq, cq), nm2 = make_float2(nm, nm);
+      const float c = __fmul_rn(ksj, cq);
+      const float nbias = -__fadd_rn(__fmul_rn(12582912.0f, c), __fmul_rn(m_new, cq));
+      const float2 c2 = make_float2(c, c), nb2 = make_float2(nbias, nbias);
       const uint32_t p_cols = tmem + lane_base + kAttColP + b * 64;
-      const float2 bs2 = partial ? att_weights<true>(sr, cq2, nm2, nvalid, p_cols)
-                                 : att_weights<false>(sr, cq2, nm2, nvalid, p_cols);
+      const float2 bs2 = partial ? att_weights<true>(sr, c2, nb2, nvalid, p_cols)
+                                 : att_weights<false>(sr, c2, nb2, nvalid, p_cols);
       if (__ballot_sync(0xFFFFFFFFu, need) != 0u && j > 0) {
         // O holds P.V of blocks < j relative to m_used: rescale it once P_{j-1} V_{j-1} has
         // landed (P_j V_j waits for this block's P)

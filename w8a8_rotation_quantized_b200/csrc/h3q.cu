@@ -471,11 +471,12 @@ struct AttLayout {
 AttLayout att_layout(int64_t S, int64_t H) {
   AttLayout l{};
   const size_t codes = size_t(H) * S * 128, scales = size_t(H) * S * 4, vt = size_t(H) * 128 * S * 2;
+  const size_t key_scales = size_t(H) * ((S + 127) / 128) * 4;  // one per block of 128 keys
   l.qq = 0;
   l.kq = align256(l.qq + codes);
   l.qs = align256(l.kq + codes);
   l.ks = align256(l.qs + scales);
-  l.vt = align256(l.ks + scales);
+  l.vt = align256(l.ks + key_scales);
   l.total = align256(l.vt + vt);
   return l;
 }
@@ -500,7 +501,7 @@ h3q_status h3q_attention_prep(const void* q, const void* k, const void* v, int64
   if (!qq || !qs || !kq || !ks || !vt || !aligned16(qq) || !aligned16(qs) || !aligned16(kq) || !aligned16(ks) ||
       !aligned16(vt))
     return H3Q_ERR_INVALID_ARG;
-  const dim3 grid(static_cast<unsigned>((S + 63) / 64), static_cast<unsigned>(H));
+  const dim3 grid(static_cast<unsigned>((S + 127) / 128), static_cast<unsigned>(H));
   h3q::attn_prep_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q),
                                                   static_cast<const __nv_bfloat16*>(k),
                                                   static_cast<const __nv_bfloat16*>(v), static_cast<int>(S), ld, qq,
