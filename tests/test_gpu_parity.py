@@ -59,7 +59,10 @@ def assert_bf16_close(got, want, where):
                                  # (values parked in tensor memory, two work items in flight, row
                                  # maxima in tagged buffers): 3 rows per item at K = 5376, so 8194
                                  # leaves a last item of one row; K = 10752 takes the searched shape
-                                 (8192, 5376), (8194, 5376), (8195, 10752)])
+                                 (8192, 5376), (8194, 5376), (8195, 10752),
+                                 # the searched shapes of that kernel for other row lengths: one group
+                                 # (64 rows per item), five groups, 28 groups
+                                 (8200, 256), (8193, 1280), (8192, 7168)])
 def test_rotate_quant_bitexact(h3q, cuda_device, M, K):
     bits, to_dev = _u(cuda_device)
     f = synth.column_factors(K, synth.outlier_columns(0, 4, K, max(1, K // 100)), 50.0)
