@@ -144,7 +144,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // the end (last block only) are set to -inf. Returns the largest F of the row.
 template <bool kMasked>
 __device__ __forceinline__ float att_raw_max(uint32_t (&sr)[4][32], int nvalid) {
-  float mx = -INFINITY;
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four chains, combined at the end
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -160,10 +160,10 @@ __device__ __forceinline__ float att_raw_max(uint32_t (&sr)[4][32], int nvalid) 
             sr[c][k0 + e] = __float_as_uint(-INFINITY);
           }
       }
-      mx = att_max3(mx, att_max3(sc[0], sc[1], sc[2]), sc[3]);
+      mx[c] = att_max3(mx[c], att_max3(sc[0], sc[1], sc[2]), sc[3]);
     }
   }
-  return mx;
+  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
 // P_k = 2^(F_k c - b) as bf16 pairs (lower key in the low half) into the 64 P
@@ -176,7 +176,8 @@ __device__ __forceinline__ float att_raw_max(uint32_t (&sr)[4][32], int nvalid) 
 template <bool kMasked>
 __device__ __forceinline__ float2 att_weights(const uint32_t (&sr)[4][32], float2 c2, float2 nb2, int nvalid,
                                               uint32_t p_cols) {
-  float2 bs2 = make_float2(0.0f, 0.0f);
+  float2 bs[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                  make_float2(0.0f, 0.0f)};  // four partial sums, so the additions do not form one chain
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     uint32_t w[32];
@@ -191,11 +192,11 @@ __device__ __forceinline__ float2 att_weights(const uint32_t (&sr)[4][32], float
         if (k0 + 1 >= nvalid) p1 = 0.0f;
       }
       w[e] = pack_bf16x2(p0, p1);
-      bs2 = __fadd2_rn(bs2, make_float2(p0, p1));
+      bs[e & 3] = __fadd2_rn(bs[e & 3], make_float2(p0, p1));
     }
     tmem_st32(p_cols + 32 * hh, w);
   }
-  return bs2;
+  return __fadd2_rn(__fadd2_rn(bs[0], bs[1]), __fadd2_rn(bs[2], bs[3]));
 }
 
 // ---------------------------------------------------------------- prep
