@@ -485,8 +485,11 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         m_used = mp;
       }
     };
+    float ks_next = set < nb ? __ldg(p.ks + int64_t(h) * nb + set) : 0.0f;
     for (int j = set; j < nb; j += 2) {
-      const int b = j & 1, vst = j % kAttVStages;
+      const int b = j & 1;
+      const float ksj = ks_next;  // loaded one block ahead: its latency stays off the score path
+      if (j + 2 < nb) ks_next = __ldg(p.ks + int64_t(h) * nb + j + 2);
       if (!(ok = wait_all(&s_full[b], static_cast<uint32_t>((j >> 1) & 1)))) break;
       tc_fence_after();
       uint32_t sr[4][32];
@@ -500,8 +503,6 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       // s' * cq, cq = qs_i log2(e) / sqrt(128) >= 0, so maxima can be taken on s', and
       // on the raw scores F = 1.5 * 2^23 + acc (ks_j >= 0). Keys past the end (last
       // block only) are masked.
-      if (!(ok = wait_all(&v_full[vst], static_cast<uint32_t>((j / kAttVStages) & 1)))) break;
-      const float ksj = __ldg(p.ks + int64_t(h) * nb + j);
       const int key0 = j * kAttBlk;
       const bool partial = key0 + kAttBlk > S;
       const int nvalid = S - key0;  // keys of the block inside the sequence (>= 8)
