@@ -118,3 +118,25 @@ def test_attention_full_size_sampled_rows(cuda_device):
     out = _run(h3q, t, S, H)
     rows = sample_indices(S, 6, np.random.default_rng(9), must=(127, 128))
     _check(out, bits, S, H, rows=rows)
+
+
+@pytest.mark.parametrize("S,H,seed", [(392, 3, 11), (136, 2, 12)])
+def test_attention_strided_views_leave_padding_untouched(cuda_device, S, H, seed):
+    """q, k, v are column slices of a matrix with padding columns past the three
+    blocks (row stride 3 H D + 64), the output a column slice of a wider NaN-filled
+    matrix: every written value is within the bound and the padding is untouched;
+    S leaves a ragged last key block of 8 keys (136) or of 8 past three blocks (392)."""
+    import w8a8_rotation_quantized_b200 as h3q
+    t, bits = _qkv(S, H, seed, cuda_device)
+    pad = 64
+    wide = torch.zeros((S, 3 * H * D + pad), dtype=torch.bfloat16, device=cuda_device)
+    wide[:, :3 * H * D] = t
+    q, k, v = wide[:, :H * D], wide[:, H * D:2 * H * D], wide[:, 2 * H * D:3 * H * D]
+    big = torch.full((S, H * D + 3 * D), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+    out = big[:, D:D + H * D]  # columns before and after the written block stay NaN
+    ws = torch.empty(h3q.h3q_attention_workspace_size(S, H), dtype=torch.uint8, device=cuda_device)
+    h3q.h3q_attention_int8(q, k, v, H, out, ws)
+    torch.cuda.synchronize()
+    assert h3q.h3q_get_device_status() == h3q.H3Q_OK
+    assert torch.isnan(big[:, :D]).all() and torch.isnan(big[:, D + H * D:]).all()
+    _check(out.contiguous(), bits, S, H)
