@@ -141,12 +141,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // The block's raw scores: the score products accumulate onto the bits of the fp32
 // value 1.5 * 2^23 (written first by one bf16 product), and |acc| <= 127^2 * 128 <
 // 2^22, so each column read as a float is F = 1.5 * 2^23 + acc exactly. Keys past
-// the end (last block only) are set to -inf. Returns the largest F of the row.
-template <bool kMasked>
-__device__ __forceinline__ float att_raw_max(uint32_t (&sr)[4][32], int nvalid) {
-  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four chains, combined at the end
+// the end (last block only) are set to -inf. Folds the 32-column chunks C0 .. C1-1
+// into the running maxima mx (one chain per chunk; the caller combines the four).
+template <bool kMasked, int C0, int C1>
+__device__ __forceinline__ void att_raw_max(uint32_t (&sr)[4][32], int nvalid, float (&mx)[4]) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = C0; c < C1; ++c) {
 #pragma unroll
     for (int e4 = 0; e4 < 8; ++e4) {
       const int k0 = 4 * e4;
@@ -163,7 +163,6 @@ __device__ __forceinline__ float att_raw_max(uint32_t (&sr)[4][32], int nvalid) 
       mx[c] = att_max3(mx[c], att_max3(sc[0], sc[1], sc[2]), sc[3]);
     }
   }
-  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
 // P_k = 2^(F_k c - b) as bf16 pairs (lower key in the low half) into the 64 P
@@ -492,21 +491,34 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       if (j + 2 < nb) ks_next = __ldg(p.ks + int64_t(h) * nb + j + 2);
       if (!(ok = wait_all(&s_full[b], static_cast<uint32_t>((j >> 1) & 1)))) break;
       tc_fence_after();
+      // Scores s' = acc * ks_j (ks_j the key block's scale); the log2-domain score is
+      // s' * cq, cq = qs_i log2(e) / sqrt(128) >= 0, so maxima can be taken on s', and
+      // on the raw scores F = 1.5 * 2^23 + acc (ks_j >= 0). Keys past the end (last
+      // block only) are masked. The row is read in two halves: the maximum of the first
+      // runs while the second is in flight.
+      const int key0 = j * kAttBlk;
+      const bool partial = key0 + kAttBlk > S;
+      const int nvalid = S - key0;  // keys of the block inside the sequence (>= 8)
       uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + kAttColS + b * kAttBlk + 32 * c, sr[c]);
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      tmem_ld32(tmem + lane_base + kAttColS + b * kAttBlk, sr[0]);
+      tmem_ld32(tmem + lane_base + kAttColS + b * kAttBlk + 32, sr[1]);
+      tmem_ld_wait();
+      tmem_ld32(tmem + lane_base + kAttColS + b * kAttBlk + 64, sr[2]);
+      tmem_ld32(tmem + lane_base + kAttColS + b * kAttBlk + 96, sr[3]);
+      if (partial)
+        att_raw_max<true, 0, 2>(sr, nvalid, mx4);
+      else
+        att_raw_max<false, 0, 2>(sr, nvalid, mx4);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[b]);  // S_{j+2} may now be written into buffer b
-      // Scores s' = acc * ks_j (ks_j the key block's scale); the log2-domain score is
-      // s' * cq, cq = qs_i log2(e) / sqrt(128) >= 0, so maxima can be taken on s', and
-      // on the raw scores F = 1.5 * 2^23 + acc (ks_j >= 0). Keys past the end (last
-      // block only) are masked.
-      const int key0 = j * kAttBlk;
-      const bool partial = key0 + kAttBlk > S;
-      const int nvalid = S - key0;  // keys of the block inside the sequence (>= 8)
-      const float f_max = partial ? att_raw_max<true>(sr, nvalid) : att_raw_max<false>(sr, nvalid);
+      if (partial)
+        att_raw_max<true, 2, 4>(sr, nvalid, mx4);
+      else
+        att_raw_max<false, 2, 4>(sr, nvalid, mx4);
+      const float f_max = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const float mx = __fmul_rn(__fsub_rn(f_max, 12582912.0f), ksj);
       if (j > 0) {  // the maximum after block j-1, published by the other set
         if (!(ok = wait_all(&mx_full[(j - 1) & 1], static_cast<uint32_t>(((j - 1) >> 1) & 1)))) break;
