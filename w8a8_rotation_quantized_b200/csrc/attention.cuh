@@ -199,96 +199,166 @@ __device__ __forceinline__ float2 att_weights(const uint32_t (&sr)[4][32], float
 }
 
 // ---------------------------------------------------------------- prep
-// Block (tile of 128 tokens = one key block, head h), 256 threads. Q rows: one
-// warp per token (4 elements per lane), a scale per token. K: the tile's max|x|
-// over its keys and dimensions gives the block's one scale, then each key row is
-// quantized with it (read again, from L1/L2). V: staged in shared memory and
-// written transposed.
-__device__ __forceinline__ void att_load4(const __nv_bfloat16* src, float (&x)[4]) {
-  const uint2 w = *reinterpret_cast<const uint2*>(src);
-  x[0] = __uint_as_float(w.x << 16);
-  x[1] = __uint_as_float(w.x & 0xFFFF0000u);
-  x[2] = __uint_as_float(w.y << 16);
-  x[3] = __uint_as_float(w.y & 0xFFFF0000u);
-}
-
-// Four int8 codes clamp(rne(x / s)) packed in a word (0 where s = 0).
-__device__ __forceinline__ uint32_t att_codes4(const float (&x)[4], float s) {
-  uint32_t packed = 0;
+// Block (tile of 128 tokens = one key block, head h), 256 threads. Every row of the
+// tile (a token's 128 values of q, k or v for head h, 256 bytes) is read as sixteen
+// 16-byte chunks, thread t taking chunks t + 256 n (n = 0..7): row (t + 256 n) / 16,
+// chunk t % 16, so a row's chunks sit in sixteen consecutive lanes. Q: the row's
+// max|x| by a 16-lane reduction, a scale per token. K: the tile's max|x| over its keys
+// and dimensions gives the block's one scale. V: the chunks go to shared memory and
+// leave transposed, each thread writing 16-byte runs of 8 tokens of one V^T row.
+__device__ __forceinline__ void att_unpack8(const uint4& w, float (&x)[8]) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    float r = 0.0f;
-    if (s != 0.0f) r = fminf(fmaxf(rintf(__fdiv_rn(x[e], s)), -127.0f), 127.0f);
-    packed |= (static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu) << (8 * e);
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(u[i] << 16);
+    x[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
   }
-  return packed;
 }
 
-__global__ void __launch_bounds__(256) attn_prep_kernel(const __nv_bfloat16* __restrict__ q,
+// Eight int8 codes clamp(rne(x / s)) in two words, element 0 in the low byte (0 where
+// s = 0); s = RN(max|x| / 127) over a set that holds these x, so |x / s| < 128.
+// rs = RN(1 / s). Fast path, as in the rotate+quantize kernel: the candidate n =
+// rne(x rs) from one FMA onto 1.5 * 2^23 (the code is then the low byte of its bits)
+// and the residual r = RN(x - n s) from another; |r| <= RN(s (1/2 - 2^-16)) puts x / s
+// within 1/2 - 2^-16 + 2^-24 of n while RN(x / s) is within 2^-18 of x / s, so n is the
+// code of the IEEE quotient. Otherwise (x / s near a half-integer), and for scales
+// below 2^-100 (whose reciprocal leaves the fp32 range), the eight codes come from the
+// IEEE quotients themselves.
+__device__ __forceinline__ uint2 att_codes8(const float (&x)[8], float s, float rs) {
+  uint32_t u[8];
+  float worst = 0.0f;
+  const float t = __fmul_rn(s, 0.4999847412109375f);  // 1/2 - 2^-16
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float c = __fmaf_rn(x[e], rs, 12582912.0f);
+    const float n = __fsub_rn(c, 12582912.0f);
+    worst = fmaxf(worst, fabsf(__fmaf_rn(-n, s, x[e])));
+    u[e] = __float_as_uint(c);
+  }
+  if (worst > t || s < 0x1p-100f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float r = s != 0.0f ? fminf(fmaxf(rintf(__fdiv_rn(x[e], s)), -127.0f), 127.0f) : 0.0f;
+      u[e] = static_cast<uint32_t>(static_cast<int>(r));
+    }
+  }
+  return make_uint2(__byte_perm(__byte_perm(u[0], u[1], 0x0040), __byte_perm(u[2], u[3], 0x0040), 0x5410),
+                    __byte_perm(__byte_perm(u[4], u[5], 0x0040), __byte_perm(u[6], u[7], 0x0040), 0x5410));
+}
+
+__device__ __forceinline__ float att_absmax8(const float (&x)[8]) {
+  float a = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[e]));
+  return a;
+}
+
+constexpr int kAttPrepPitch = kAttD / 2 + 1;  // words per staged V row (128 bf16 + one pad word)
+
+__global__ void __launch_bounds__(256, 2) attn_prep_kernel(const __nv_bfloat16* __restrict__ q,
                                                         const __nv_bfloat16* __restrict__ k,
                                                         const __nv_bfloat16* __restrict__ v, int S, int64_t ld,
                                                         int8_t* __restrict__ qq, float* __restrict__ qs,
                                                         int8_t* __restrict__ kq, float* __restrict__ ks,
                                                         __nv_bfloat16* __restrict__ vt) {
-  __shared__ uint16_t tile[kAttBlk][kAttD + 2];  // +2 halves: column reads spread over banks
+  __shared__ uint32_t tile[kAttBlk * kAttPrepPitch];  // V rows (token-major), bf16 pairs
   __shared__ float warp_max[8];
   const int h = blockIdx.y;
   const int t0 = blockIdx.x * kAttBlk;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Q: a scale per token
-  for (int t = warp; t < kAttBlk; t += 8) {
-    const int i = t0 + t;
-    if (i >= S) break;
-    float x[4];
-    att_load4(q + int64_t(i) * ld + h * kAttD + 4 * lane, x);
-    float a = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+  const int cc = threadIdx.x & 15;  // 16-byte chunk of the row: dimensions 8 cc .. 8 cc + 7
+  uint4 wq[8], wk[8];  // raw bf16 chunks: every load of Q and K in flight at once
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  for (int n = 0; n < 8; ++n) {
+    const int row = (threadIdx.x >> 4) + 16 * n;
+    const int i = t0 + row;
+    wq[n] = wk[n] = make_uint4(0u, 0u, 0u, 0u);
+    if (i < S) {
+      const int64_t off = int64_t(i) * ld + h * kAttD + 8 * cc;
+      wq[n] = *reinterpret_cast<const uint4*>(q + off);
+      wk[n] = *reinterpret_cast<const uint4*>(k + off);
+    }
+  }
+  // Q: a scale per token
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    const int row = (threadIdx.x >> 4) + 16 * n;
+    const int i = t0 + row;
+    float x[8];
+    att_unpack8(wq[n], x);
+    float a = att_absmax8(x);
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
     const float sq = __fdiv_rn(a, 127.0f);
-    const int64_t row = int64_t(h) * S + i;
-    *reinterpret_cast<uint32_t*>(qq + row * kAttD + 4 * lane) = att_codes4(x, sq);
-    if (lane == 0) qs[row] = sq;
+    const float rq = sq != 0.0f ? __frcp_rn(sq) : 0.0f;
+    if (i < S) {
+      const int64_t r = int64_t(h) * S + i;
+      *reinterpret_cast<uint2*>(qq + r * kAttD + 8 * cc) = att_codes8(x, sq, rq);
+      if (cc == 0) qs[r] = sq;
+    }
   }
   // K: one scale for the tile's keys
   float a = 0.0f;
-  for (int t = warp; t < kAttBlk; t += 8) {
-    const int i = t0 + t;
-    if (i >= S) break;
-    float x[4];
-    att_load4(k + int64_t(i) * ld + h * kAttD + 4 * lane, x);
-    a = fmaxf(a, fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))));
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    float x[8];
+    att_unpack8(wk[n], x);
+    a = fmaxf(a, att_absmax8(x));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
   if (lane == 0) warp_max[warp] = a;
+  // V rows into shared memory (loaded while the K maximum is combined)
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    const int row = (threadIdx.x >> 4) + 16 * n;
+    const int i = t0 + row;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (i < S) w = *reinterpret_cast<const uint4*>(v + int64_t(i) * ld + h * kAttD + 8 * cc);
+    uint32_t* dst = tile + row * kAttPrepPitch + 4 * cc;
+    dst[0] = w.x;
+    dst[1] = w.y;
+    dst[2] = w.z;
+    dst[3] = w.w;
+  }
   __syncthreads();
 #pragma unroll
   for (int w = 0; w < 8; ++w) a = fmaxf(a, warp_max[w]);
   const float sk = __fdiv_rn(a, 127.0f);
+  const float rk = sk != 0.0f ? __frcp_rn(sk) : 0.0f;
   if (threadIdx.x == 0) ks[int64_t(h) * gridDim.x + blockIdx.x] = sk;
-  for (int t = warp; t < kAttBlk; t += 8) {
-    const int i = t0 + t;
-    if (i >= S) break;
-    float x[4];
-    att_load4(k + int64_t(i) * ld + h * kAttD + 4 * lane, x);
-    *reinterpret_cast<uint32_t*>(kq + (int64_t(h) * S + i) * kAttD + 4 * lane) = att_codes4(x, sk);
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    const int row = (threadIdx.x >> 4) + 16 * n;
+    const int i = t0 + row;
+    float x[8];
+    att_unpack8(wk[n], x);
+    if (i < S) *reinterpret_cast<uint2*>(kq + (int64_t(h) * S + i) * kAttD + 8 * cc) = att_codes8(x, sk, rk);
   }
-  // V tile [128 tokens][128 d] -> V^T rows h*128 + d, columns t0 .. t0+127
-  for (int e = threadIdx.x; e < kAttBlk * (kAttD / 2); e += 256) {
-    const int t = e / (kAttD / 2), d2 = e % (kAttD / 2);
-    const int i = t0 + t;
-    uint32_t w = 0;
-    if (i < S) w = *reinterpret_cast<const uint32_t*>(v + int64_t(i) * ld + h * kAttD + 2 * d2);
-    tile[t][2 * d2] = static_cast<uint16_t>(w & 0xFFFFu);
-    tile[t][2 * d2 + 1] = static_cast<uint16_t>(w >> 16);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < kAttD * (kAttBlk / 2); e += 256) {
-    const int d = e / (kAttBlk / 2), t2 = e % (kAttBlk / 2);  // tokens 2 t2, 2 t2 + 1
-    const int i = t0 + 2 * t2;
-    if (i >= S) continue;
-    const uint32_t w = uint32_t(tile[2 * t2][d]) | (uint32_t(tile[2 * t2 + 1][d]) << 16);
-    *reinterpret_cast<uint32_t*>(vt + (int64_t(h) * kAttD + d) * S + i) = w;
+  // V^T: lane l takes dimension pair p = 32 (u % 2) + l (dimensions 2p, 2p + 1) and the
+  // 8-token group g = 2 warp + u / 2 (u = 0..3); it reads word p of rows 8 g .. 8 g + 7
+  // (consecutive lanes, consecutive words: no bank conflict) and writes 8 tokens of V^T
+  // rows h*128 + 2p and h*128 + 2p + 1 as two 16-byte stores.
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int p = 32 * (u & 1) + lane;
+    const int g = 2 * warp + (u >> 1);
+    const int i0 = t0 + 8 * g;
+    if (i0 >= S) continue;  // S % 8 == 0: a group is wholly inside or outside
+    uint32_t wv[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) wv[m] = tile[(8 * g + m) * kAttPrepPitch + p];
+    uint4 lo, hi;  // dimension 2p (low halves) and 2p + 1 (high halves) of tokens i0 .. i0 + 7
+    lo.x = __byte_perm(wv[0], wv[1], 0x5410);
+    lo.y = __byte_perm(wv[2], wv[3], 0x5410);
+    lo.z = __byte_perm(wv[4], wv[5], 0x5410);
+    lo.w = __byte_perm(wv[6], wv[7], 0x5410);
+    hi.x = __byte_perm(wv[0], wv[1], 0x7632);
+    hi.y = __byte_perm(wv[2], wv[3], 0x7632);
+    hi.z = __byte_perm(wv[4], wv[5], 0x7632);
+    hi.w = __byte_perm(wv[6], wv[7], 0x7632);
+    *reinterpret_cast<uint4*>(vt + (int64_t(h) * kAttD + 2 * p) * S + i0) = lo;
+    *reinterpret_cast<uint4*>(vt + (int64_t(h) * kAttD + 2 * p + 1) * S + i0) = hi;
   }
 }
 
