@@ -178,11 +178,11 @@ __device__ __forceinline__ float2 att_weights(const uint32_t (&sr)[4][32], float
   float2 bs[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
                   make_float2(0.0f, 0.0f)};  // four partial sums, so the additions do not form one chain
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    uint32_t w[32];
+  for (int hh = 0; hh < 4; ++hh) {  // 32 keys (16 P columns) per store, so each store overlaps the next keys
+    uint32_t w[16];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int k0 = 64 * hh + 2 * e;
+    for (int e = 0; e < 16; ++e) {
+      const int k0 = 32 * hh + 2 * e;
       const float2 t = __ffma2_rn(
           make_float2(__uint_as_float(sr[k0 >> 5][k0 & 31]), __uint_as_float(sr[k0 >> 5][(k0 & 31) + 1])), c2, nb2);
       float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
@@ -193,7 +193,7 @@ __device__ __forceinline__ float2 att_weights(const uint32_t (&sr)[4][32], float
       w[e] = pack_bf16x2(p0, p1);
       bs[e & 3] = __fadd2_rn(bs[e & 3], make_float2(p0, p1));
     }
-    tmem_st32(p_cols + 32 * hh, w);
+    tmem_st16(p_cols + 16 * hh, w);
   }
   return __fadd2_rn(__fadd2_rn(bs[0], bs[1]), __fadd2_rn(bs[2], bs[3]));
 }
